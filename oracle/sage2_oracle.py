@@ -1,0 +1,388 @@
+"""CPU oracle for the SageAttention2 quantized attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py`` (its CPU-baseline / reference leg) may import this module.  The
+product path (the CUDA library and its Python binding) never calls it and shares
+no code, header, table or helper with it.
+
+What it computes.  "SageAttention2: Efficient Attention with Thorough Outlier
+Smoothing and Per-thread INT4 Quantization" (arxiv.science abstract page,
+Abstract) describes the method in four moves: Q and K are quantized to INT4 at a
+fine per-thread granularity, P~ and V to FP8, Q is smoothed to make the INT4
+QK^T accurate, and P~V is accumulated in two levels.  K smoothing (subtracting
+the token mean of K, which softmax ignores) is the "outlier smoothing" of the
+title, inherited from the predecessor "SageAttention: Accurate 8-Bit Attention"
+(ainnect.com/research/19 summary).  The method is an approximation, so this
+oracle takes its steps in that order, one function per step, with the plainest
+reading wherever the pages are silent (every reading is listed in the module
+constants and in the function docstrings):
+
+  1. k_mean            K smoothing: token mean of K per channel.
+  2. q_block_means     Q smoothing: mean of each 128-row block of Q.
+  3. quant_int4_rows   INT4 on [-7, 7], one scale per token (row).
+  4. qk_correction     the fp32 correction  qbar_blk . K_j  that Q smoothing
+                       subtracted (row constant qbar.kbar dropped).
+  5. quant_v           FP8 e4m3 V, one scale per channel.
+  6. attn_quantized    INT4 QK^T (exact integers), online softmax over 128-key
+                       tiles, P~ to e4m3 with the fixed scale 448, P~V summed
+                       per tile (inner level) then added to the running output
+                       (outer level).
+  7. attn_fp64         the unquantized reference  softmax(QK^T * sm_scale) V.
+
+Precision.  Steps 1-3 and 5 produce the payloads (the integers, codes and
+scales the kernels also produce); they are written in float32 with a fixed
+operation order so that they are reproducible bit for bit.  Steps 4, 6 and 7
+are done in float64 (exact products of the quantized values, fp64 sums).
+
+Parity pins (tests/test_oracle_*.py): e4m3 codec against the format's code
+table and torch's converter; INT4 ties and bounds; means against fp64; the
+Q-smoothing reconstruction and the K-smoothing shift invariance in fp64; the
+online-softmax/tiling path with the quantizers swapped for the identity against
+direct fp64 attention; single-tile brute force; the N=1 and uniform-attention
+closed forms.  End-to-end accuracy against the paper is "parity unpinned": the
+pages print no accuracy numbers.
+"""
+from __future__ import annotations
+
+import math
+import numpy as np
+
+BM = 128            # rows of Q per smoothing block / per attention tile
+BN = 128            # keys per attention tile (the "inner" accumulation block)
+INT4_MAX = 7        # symmetric INT4 range [-7, 7]
+E4M3_MAX = 448.0    # largest finite e4m3 value; also the fixed P~ scale
+LOG2E = 1.4426950408889634
+
+# Relative distance from an e4m3 rounding boundary inside which the rounding of
+# 448*p is treated as ambiguous: the kernel evaluates p = exp2(x - m) in fp32
+# (x built from fp32 products and sums, exp2 with ~2 ulp error), so 448*p can
+# differ from the fp64 value by up to a few 1e-5 relative; either neighbouring
+# code is then a correct result.
+AMBIG_REL = 2.0 ** -13
+
+
+def n_pad(N: int) -> int:
+    return ((N + BM - 1) // BM) * BM
+
+
+# ----------------------------------------------------------------------------
+# FP8 e4m3 ("e4m3fn": 4 exponent bits, bias 7, 3 mantissa bits, no infinity,
+# S.1111.111 is NaN, largest finite 448, smallest subnormal 2^-9).  Written from
+# the format definition; rounding is to nearest, ties to even, and values beyond
+# the largest finite magnitude saturate to +-448 (the "satfinite" behaviour).
+# ----------------------------------------------------------------------------
+
+def e4m3_value_table() -> np.ndarray:
+    """float64 value of each of the 256 codes (NaN for the two NaN codes)."""
+    vals = np.empty(256, np.float64)
+    for code in range(256):
+        s = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            vals[code] = np.nan
+        elif e == 0:
+            vals[code] = s * m * 2.0 ** -9
+        else:
+            vals[code] = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return vals
+
+
+_E4M3_VALUES = e4m3_value_table()
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Round finite values to e4m3 codes (RNE, saturating). Returns uint8."""
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    sign = (np.signbit(x)).astype(np.uint8) << 7
+    code = np.zeros(a.shape, np.int64)
+    sub = a < 2.0 ** -6
+    # subnormal range: quantum 2^-9; k = 8 rounds up into the first normal code
+    k_sub = np.rint(a * 2.0 ** 9)
+    code = np.where(sub, k_sub.astype(np.int64), code)
+    # normal range: quantum 2^(e-3) with e = floor(log2 a)
+    _, E = np.frexp(np.where(sub, 1.0, a))
+    e = E - 1
+    k = np.rint(np.ldexp(np.where(sub, 1.0, a), 3 - e))       # in [8, 16]
+    carry = k >= 16
+    e = np.where(carry, e + 1, e)
+    k = np.where(carry, 8, k)
+    code_n = ((e + 7) << 3) | (k.astype(np.int64) - 8)
+    code = np.where(sub, code, code_n)
+    code = np.where(a >= E4M3_MAX, 0x7E, code)
+    code = np.minimum(code, 0x7E)
+    return (code.astype(np.uint8) | sign).astype(np.uint8)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    return _E4M3_VALUES[np.asarray(codes, np.uint8)]
+
+
+def e4m3_round(x) -> np.ndarray:
+    """x rounded to the nearest e4m3 value (float64)."""
+    return e4m3_decode(e4m3_encode(x))
+
+
+def e4m3_ambiguity(y) -> np.ndarray:
+    """For y >= 0: |gap| between the two e4m3 neighbours if y lies within
+    AMBIG_REL (relative) of a rounding boundary, else 0."""
+    y = np.asarray(y, np.float64)
+    lo = e4m3_round(y * (1.0 - AMBIG_REL))
+    hi = e4m3_round(y * (1.0 + AMBIG_REL))
+    return np.abs(hi - lo)
+
+
+# ----------------------------------------------------------------------------
+# Step 1 - K smoothing: kbar[c] = (1/N) sum_j K[j, c].
+# Reading (fixed order, so the payloads are reproducible): float32 sums, each
+# 128-token chunk summed token by token in ascending order starting at 0, then
+# the chunk sums added one after another in chunk order starting at 0, then one
+# IEEE float32 division by N.
+# ----------------------------------------------------------------------------
+
+def k_mean(K: np.ndarray) -> np.ndarray:
+    """K: [N, d] (any float dtype; converted exactly to float32) -> [d] float32."""
+    K = np.asarray(K, np.float32)
+    N, d = K.shape
+    total = np.zeros(d, np.float32)
+    for c0 in range(0, N, BN):
+        part = np.zeros(d, np.float32)
+        for j in range(c0, min(c0 + BN, N)):
+            part = part + K[j]
+        total = total + part
+    return (total / np.float32(N)).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# Step 2 - Q smoothing: one mean per block of BM consecutive query rows.
+# Reading: float32 sum over the block's valid rows in ascending order starting
+# at 0, divided (IEEE float32) by the number of valid rows.
+# ----------------------------------------------------------------------------
+
+def q_block_means(Q: np.ndarray) -> np.ndarray:
+    """Q: [N, d] -> qbar [ceil(N/BM), d] float32."""
+    Q = np.asarray(Q, np.float32)
+    N, d = Q.shape
+    nb = (N + BM - 1) // BM
+    out = np.zeros((nb, d), np.float32)
+    for b in range(nb):
+        r0, r1 = b * BM, min(N, (b + 1) * BM)
+        acc = np.zeros(d, np.float32)
+        for i in range(r0, r1):
+            acc = acc + Q[i]
+        out[b] = acc / np.float32(r1 - r0)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Step 3 - INT4 quantization, one scale per token (per row of d channels).
+# Reading of the per-thread granularity for the Blackwell MMA layout: every
+# accumulator row (a query) and every accumulator column (a key) carries its
+# own scale.  scale = amax/7 and inv = 7/amax (float32 IEEE), q = RNE(x*inv)
+# clamped to [-7, 7]; an all-zero row gets scale 0 and q = 0.
+# ----------------------------------------------------------------------------
+
+def quant_int4_rows(X: np.ndarray):
+    """X: [n, d] float32 -> (q int8 [n, d], scale float32 [n])."""
+    X = np.asarray(X, np.float32)
+    amax = np.max(np.abs(X), axis=1)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    scale = np.where(nz, safe / np.float32(INT4_MAX), np.float32(0)).astype(np.float32)
+    inv = (np.float32(INT4_MAX) / safe).astype(np.float32)
+    y = (X * inv[:, None]).astype(np.float32)
+    q = np.clip(np.rint(y), -INT4_MAX, INT4_MAX).astype(np.int8)
+    q[~nz] = 0
+    return q, scale
+
+
+def smooth_quant_qk(Q: np.ndarray, K: np.ndarray):
+    """One head. Q, K: [N, d]. Returns the padded payloads:
+    q_i4 [Np, d] int8, q_scale [Np] f32, q_mean [Np/BM, d] f32,
+    k_i4 [Np, d] int8, k_scale [Np] f32, k_mean [d] f32.  Rows >= N are 0."""
+    Q = np.asarray(Q, np.float32)
+    K = np.asarray(K, np.float32)
+    N, d = Q.shape
+    Np = n_pad(N)
+    kbar = k_mean(K)
+    Ks = (K - kbar[None, :]).astype(np.float32)
+    qbar = q_block_means(Q)
+    Qs = (Q - np.repeat(qbar, BM, axis=0)[:N]).astype(np.float32)
+    q_i4 = np.zeros((Np, d), np.int8)
+    k_i4 = np.zeros((Np, d), np.int8)
+    q_scale = np.zeros(Np, np.float32)
+    k_scale = np.zeros(Np, np.float32)
+    q_i4[:N], q_scale[:N] = quant_int4_rows(Qs)
+    k_i4[:N], k_scale[:N] = quant_int4_rows(Ks)
+    return dict(q_i4=q_i4, q_scale=q_scale, q_mean=qbar, k_i4=k_i4,
+                k_scale=k_scale, k_mean=kbar)
+
+
+# ----------------------------------------------------------------------------
+# Step 4 - Q-smoothing correction.  Q K_s^T = Q_s K_s^T + qbar_blk K_s^T; the
+# second term is added back in floating point.  Reading: it is formed with the
+# raw K (qbar . K_j); the difference qbar.kbar is constant along each row and
+# softmax ignores it.
+# ----------------------------------------------------------------------------
+
+def qk_correction(q_mean: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """q_mean [nb, d] f32, K [N, d] -> C [nb, Np] float64 (0 beyond N)."""
+    K = np.asarray(K, np.float64)
+    N = K.shape[0]
+    C = np.zeros((q_mean.shape[0], n_pad(N)), np.float64)
+    C[:, :N] = np.asarray(q_mean, np.float64) @ K.T
+    return C
+
+
+# ----------------------------------------------------------------------------
+# Step 5 - V to FP8 e4m3, one scale per channel over all tokens.
+# Reading: sv = amax/448, inv = 448/amax (float32 IEEE), code = e4m3(V*inv)
+# rounded to nearest even with saturation; an all-zero channel gets sv = 0.
+# The codes are stored transposed, [d, Np] (token-contiguous), pad tokens 0.
+# ----------------------------------------------------------------------------
+
+def quant_v(V: np.ndarray):
+    """V: [N, d] -> (v_t codes uint8 [d, Np], v_scale f32 [d])."""
+    V = np.asarray(V, np.float32)
+    N, d = V.shape
+    amax = np.max(np.abs(V), axis=0)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    sv = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(0)).astype(np.float32)
+    inv = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    y = (V * inv[None, :]).astype(np.float32)
+    codes = e4m3_encode(y)
+    codes[:, ~nz] = 0
+    vt = np.zeros((d, n_pad(N)), np.uint8)
+    vt[:, :N] = codes.T
+    return vt, sv
+
+
+# ----------------------------------------------------------------------------
+# Step 6 - attention over the quantized payloads.
+# ----------------------------------------------------------------------------
+
+def qk_int(q_i4: np.ndarray, k_i4: np.ndarray) -> np.ndarray:
+    """Exact integer Q^ K^T (int64): the INT4 matrix product."""
+    # fp64 matmul of small integers is exact (|sum| <= 49*d << 2^53)
+    return (np.asarray(q_i4, np.float64) @ np.asarray(k_i4, np.float64).T).astype(np.int64)
+
+
+def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
+                   q_blocks=None, quantize: bool = True):
+    """Online-softmax attention of one head over its payloads.
+
+    p: dict with q_i4, q_scale, k_i4, k_scale, C (qk_correction), v_t, v_scale
+       (with quantize=False: 'q_s' / 'k_s' float rows replace q_i4*q_scale /
+       k_i4*k_scale and 'v' [N, d] replaces the e4m3 V; P~ is not rounded).
+    q_blocks: iterable of 128-row query block indices to compute (default all).
+    Returns (O [rows, d] float64, amb [rows, d] float64, rows index array).
+
+    Per query block and for key tiles in ascending order (causal: tiles above
+    the diagonal skipped; masked scores are -inf), with L = sm_scale*log2(e):
+        x    = (sq_i sk_j S_ij + C_blk,j) * L
+        m'   = max(m, rowmax x);   alpha = exp2(m - m')   (0 when m = -inf)
+        p    = exp2(x - m');       l = alpha*l + sum_j p  (p before rounding)
+        P~   = e4m3(448 p)
+        inner= P~ . V~  over this tile only              (inner level)
+        acc  = alpha*acc + inner                          (outer level)
+    then O = acc * sv / (448 l).  'amb' bounds what a different but equally
+    correct rounding of ambiguous 448p values (see AMBIG_REL) can change.
+    """
+    Np = n_pad(N)
+    nb = Np // BM
+    L = sm_scale * LOG2E
+    if quantize:
+        qv = np.asarray(p["q_i4"], np.float64)
+        kv = np.asarray(p["k_i4"], np.float64)
+        sq = np.asarray(p["q_scale"], np.float64)
+        sk = np.asarray(p["k_scale"], np.float64)
+        vdec = e4m3_decode(p["v_t"]).T            # [Np, d] decoded codes
+        sv = np.asarray(p["v_scale"], np.float64)
+    else:
+        qv = np.zeros((Np, p["q_s"].shape[1])); qv[:N] = p["q_s"]
+        kv = np.zeros((Np, p["k_s"].shape[1])); kv[:N] = p["k_s"]
+        sq = np.ones(Np); sk = np.ones(Np)
+        vdec = np.zeros((Np, p["v"].shape[1])); vdec[:N] = p["v"]
+        sv = np.ones(vdec.shape[1])
+    C = np.asarray(p["C"], np.float64)
+    d = vdec.shape[1]
+    blocks = range(nb) if q_blocks is None else q_blocks
+    outs, ambs, rows = [], [], []
+    for b in blocks:
+        r = np.arange(b * BM, min((b + 1) * BM, N))
+        if r.size == 0:
+            continue
+        m = np.full(r.size, -np.inf)
+        l = np.zeros(r.size)
+        acc = np.zeros((r.size, d))
+        amb = np.zeros((r.size, d))
+        last = b if causal else nb - 1
+        for t in range(last + 1):
+            c = np.arange(t * BN, (t + 1) * BN)
+            S = qv[r] @ kv[c].T                                   # exact
+            x = (sq[r, None] * sk[None, c] * S + C[b][c][None, :]) * L
+            mask = c[None, :] >= N
+            if causal:
+                mask = mask | (c[None, :] > r[:, None])
+            x = np.where(mask, -np.inf, x)
+            m_new = np.maximum(m, x.max(axis=1))
+            alpha = np.where(np.isneginf(m), 0.0, np.exp2(m - m_new))
+            pt = np.exp2(x - m_new[:, None])
+            l = alpha * l + pt.sum(axis=1)
+            if quantize:
+                ph = e4m3_round(E4M3_MAX * pt)
+                gap = e4m3_ambiguity(E4M3_MAX * pt)
+            else:
+                ph, gap = pt, np.zeros_like(pt)
+            inner = ph @ vdec[c]                                  # inner level
+            acc = alpha[:, None] * acc + inner                    # outer level
+            amb = alpha[:, None] * amb + gap @ np.abs(vdec[c])
+            m = m_new
+        scale = E4M3_MAX if quantize else 1.0
+        outs.append(acc * sv[None, :] / (scale * l[:, None]))
+        ambs.append(amb * sv[None, :] / (scale * l[:, None]))
+        rows.append(r)
+    if not outs:
+        return np.zeros((0, d)), np.zeros((0, d)), np.zeros(0, np.int64)
+    return np.concatenate(outs), np.concatenate(ambs), np.concatenate(rows)
+
+
+# ----------------------------------------------------------------------------
+# Step 7 - the unquantized reference.
+# ----------------------------------------------------------------------------
+
+def attn_fp64(Q, K, V, causal: bool, sm_scale: float, rows=None) -> np.ndarray:
+    """softmax(Q K^T sm_scale) V in float64, top-left causal mask (j <= i)."""
+    Q = np.asarray(Q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    N = Q.shape[0]
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    s = (Q[rows] @ K.T) * sm_scale
+    if causal:
+        s = np.where(np.arange(N)[None, :] > rows[:, None], -np.inf, s)
+    s = s - s.max(axis=1, keepdims=True)
+    w = np.exp(s)
+    return (w @ V) / w.sum(axis=1, keepdims=True)
+
+
+# ----------------------------------------------------------------------------
+# The whole pipeline for one head.
+# ----------------------------------------------------------------------------
+
+def sage2_head(Q, K, V, causal: bool, sm_scale: float | None = None, q_blocks=None):
+    """Steps 1-6 for one head.  Q, K, V: [N, d] (fp16/bf16 values as float32).
+    Returns (payload dict, O rows, amb rows, row index)."""
+    Q = np.asarray(Q, np.float32)
+    K = np.asarray(K, np.float32)
+    V = np.asarray(V, np.float32)
+    N, d = Q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    pay = smooth_quant_qk(Q, K)
+    pay["C"] = qk_correction(pay["q_mean"], K)
+    pay["v_t"], pay["v_scale"] = quant_v(V)
+    O, amb, rows = attn_quantized(pay, N, causal, sm_scale, q_blocks=q_blocks)
+    return pay, O, amb, rows
