@@ -1,0 +1,148 @@
+/*
+ * sage2.h - C ABI of the B200 (sm_100a) SageAttention2 quantized attention
+ * forward pass:  O = softmax(Q K^T * sm_scale) V  computed with smoothed INT4
+ * Q/K, FP8 (e4m3) P~/V and two-level P~V accumulation.
+ *
+ * The method follows "SageAttention2: Efficient Attention with Thorough
+ * Outlier Smoothing and Per-thread INT4 Quantization" (arxiv.science abstract
+ * page, Abstract): INT4 (Q, K) at a per-thread granularity, FP8 (P~, V),
+ * smoothing of Q for the INT4 QK^T, two-level accumulation for the FP8 P~V.
+ * K smoothing (token mean removed) is the "outlier smoothing" of the title.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major ("HND"): q, k, v, o are [B, H, N, d].
+ *  - d is 64 or 128.  N >= 1.  B*H >= 1.  Np = ceil(N/128)*128, NB = Np/128.
+ *  - All pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *    The library never frees caller memory.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default
+ *    stream) and returns before the GPU work ends.  Arguments are validated on
+ *    the host before anything is launched; a non-OK status means nothing was
+ *    launched (except SAGE2_ERR_CUDA, which reports a failed launch).
+ *  - No C++ exception crosses the ABI.
+ *  - Causal masking is top-left aligned: query i sees keys j <= i.
+ *
+ * Payload layouts (the quantized intermediates, all on the device)
+ * ----------------------------------------------------------------
+ *  q_i4   int8  [B,H,Np,d]   INT4 values in [-7,7] of Q - qbar_block, rows >= N are 0
+ *  q_scale f32  [B,H,Np]     per-token scale amax/7 (0 for an all-zero row / pad)
+ *  q_mean f32   [B,H,NB,d]   mean of each 128-row block of Q (valid rows only)
+ *  k_i4   int8  [B,H,Np,d]   INT4 values of K - kbar, rows >= N are 0
+ *  k_scale f32  [B,H,Np]     per-token scale
+ *  k_mean f32   [B,H,d]      token mean of K
+ *  qk_corr f32  [B,H,NB,Np]  q_mean[blk] . K[j] (raw K), 0 for j >= N
+ *  v_fp8_t u8   [B,H,d,Np]   e4m3 codes of V * 448/amax_c, TRANSPOSED (token-contiguous)
+ *  v_scale f32  [B,H,d]      per-channel scale amax_c/448
+ */
+#ifndef SAGE2_H_
+#define SAGE2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* sage2_stream_t;
+
+typedef enum {
+  SAGE2_OK = 0,
+  SAGE2_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad dtype   */
+  SAGE2_ERR_UNSUPPORTED = 2, /* d not in {64,128}, size beyond int32 indexing */
+  SAGE2_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned              */
+  SAGE2_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed   */
+  SAGE2_ERR_NO_MEM = 5,      /* workspace allocation failed                   */
+  SAGE2_ERR_TIMEOUT = 6      /* a kernel's bounded wait ran out (device word) */
+} sage2_status;
+
+typedef enum { SAGE2_F16 = 0, SAGE2_BF16 = 1, SAGE2_F32 = 2 } sage2_dtype;
+
+/*
+ * Smoothing + INT4 quantization of Q and K, and the Q-smoothing correction.
+ * (Abstract: INT4 (Q,K) at per-thread granularity; "a method to smooth Q".)
+ *   q, k      : [B,H,N,d] in `dtype` (SAGE2_F16 or SAGE2_BF16).
+ *   outputs   : q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr as in the
+ *               payload table above (caller-allocated, fully overwritten,
+ *               including the pad rows/columns).
+ * Semantics: kbar = fixed-order fp32 token mean of K (128-token chunks summed
+ * in token order, chunk sums in chunk order, one fp32 division by N); qbar per
+ * 128-row block likewise over the valid rows; x = fp32(X) - mean;
+ * scale = amax/7; q = clamp(rint(x * (7/amax)), -7, 7) (all fp32, RNE).
+ * qk_corr[blk][j] = sum_c q_mean[blk][c] * K[j][c], fp32.
+ */
+sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int B, int H, int N,
+                                   int d, int8_t* q_i4, float* q_scale, float* q_mean,
+                                   int8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
+                                   sage2_stream_t stream);
+
+/*
+ * FP8 e4m3 quantization of V with one scale per channel (Abstract: FP8 V).
+ *   v        : [B,H,N,d] in `dtype`.
+ *   v_fp8_t  : [B,H,d,Np] e4m3 codes, token-contiguous; pad tokens are 0.
+ *   v_scale  : [B,H,d] = amax_c/448 (0 for an all-zero channel).
+ * Codes are RNE of fp32(V * (448/amax_c)) with saturation to +-448.
+ */
+sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d,
+                           uint8_t* v_fp8_t, float* v_scale, sage2_stream_t stream);
+
+/*
+ * Attention over the quantized payloads (the fused tcgen05 kernel alone).
+ * (Abstract: INT4 QK^T; FP8 P~V with two-level accumulation.)
+ *   o       : [B,H,N,d] written in `o_dtype` (SAGE2_F16, SAGE2_BF16 or SAGE2_F32).
+ *   causal  : 0 or 1.   sm_scale : softmax scale (> 0, finite).
+ * Per 128-key tile, in ascending order, with L = sm_scale*log2(e):
+ *   x = (q_scale_i*k_scale_j*S_ij + qk_corr[blk(i)][j]) * L,  S = q_i4 . k_i4 (s32)
+ *   running max m, p = exp2(x - m), l += p, P~ = e4m3(448 p),
+ *   inner = P~ . V~ over the tile (fresh fp32 accumulator),
+ *   acc = alpha*acc + inner (alpha = exp2(m_old - m_new));  O = acc*v_scale/(448 l).
+ */
+sage2_status sage2_attn_fwd_quantized(const int8_t* q_i4, const float* q_scale,
+                                      const int8_t* k_i4, const float* k_scale,
+                                      const float* qk_corr, const uint8_t* v_fp8_t,
+                                      const float* v_scale, void* o, int o_dtype, int B, int H,
+                                      int N, int d, int causal, float sm_scale,
+                                      sage2_stream_t stream);
+
+/*
+ * The whole forward pass: smoothing + quantization of Q, K, V, the correction
+ * and the attention kernel, with the payloads in a workspace that the library
+ * takes from its own stream-ordered memory pool and returns on `stream`
+ * (sage2_workspace_bytes() tells how much).
+ *   q, k, v : [B,H,N,d] in `dtype` (SAGE2_F16 / SAGE2_BF16);  o in `o_dtype`.
+ * Returns SAGE2_ERR_NO_MEM when the pool cannot provide the workspace.
+ */
+sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int N, int d, int dtype, int o_dtype, int causal, float sm_scale,
+                            sage2_stream_t stream);
+
+/* Bytes of workspace sage2_attn_fwd takes for this problem (0 on bad sizes). */
+size_t sage2_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Test entry: the raw integer products S = q_i4 . k_i4^T of every 128x128
+ * tile, through the same TMA + tcgen05 kind::i8 path as the attention kernel.
+ *   s_out : int32 [B,H,Np,Np] (caller-allocated).
+ */
+sage2_status sage2_debug_qk_s32(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int N,
+                                int d, int32_t* s_out, sage2_stream_t stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device error word that
+ * kernels set instead of trapping.  SAGE2_ERR_TIMEOUT if a bounded wait ran
+ * out, SAGE2_ERR_CUDA on a sticky CUDA error, else SAGE2_OK.
+ */
+sage2_status sage2_check_device_error(sage2_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char* sage2_status_string(sage2_status status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int sage2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE2_H_ */

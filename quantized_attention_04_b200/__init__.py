@@ -1,0 +1,202 @@
+"""Python binding of libsage2 (the B200 SageAttention2 forward pass).
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libsage2.so`` (built in-tree by ``python -m quantized_attention_04_b200.build``),
+called through its C ABI (include/sage2.h).  Importing works without a GPU;
+calling any compute entry point without the built library raises.
+
+The functions keep the C names.  Tensors are torch CUDA tensors; outputs are
+allocated with torch on the input's device and every call is enqueued on
+torch's current stream of that device.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "sage2_smooth_quant_qk", "sage2_quant_v", "sage2_attn_fwd_quantized", "sage2_attn_fwd",
+    "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
+    "sage2_status_string", "sage2_version", "attn", "Sage2Error", "lib", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage2.so")
+F16, BF16, F32 = 0, 1, 2
+_DT = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+STATUS = {0: "SAGE2_OK", 1: "SAGE2_ERR_INVALID_ARG", 2: "SAGE2_ERR_UNSUPPORTED",
+          3: "SAGE2_ERR_MISALIGNED", 4: "SAGE2_ERR_CUDA", 5: "SAGE2_ERR_NO_MEM",
+          6: "SAGE2_ERR_TIMEOUT"}
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SIGS = {
+    "sage2_smooth_quant_qk": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "sage2_quant_v": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sage2_attn_fwd_quantized": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sage2_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sage2_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "sage2_debug_qk_s32": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
+    "sage2_check_device_error": (_I, [_P]),
+    "sage2_status_string": (ctypes.c_char_p, [_I]),
+    "sage2_version": (_I, []),
+}
+
+
+class Sage2Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} "
+                         f"({lib().sage2_status_string(status).decode()})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsage2.so; raises ImportError if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m quantized_attention_04_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise Sage2Error(fn, status)
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dims(x: torch.Tensor):
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    if not x.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return x.shape
+
+
+def n_pad(N: int) -> int:
+    return (N + 127) // 128 * 128
+
+
+def sage2_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().sage2_workspace_bytes(B, H, N, d))
+
+
+def sage2_status_string(status: int) -> str:
+    return lib().sage2_status_string(status).decode()
+
+
+def sage2_version() -> int:
+    return int(lib().sage2_version())
+
+
+def sage2_check_device_error(device=None) -> int:
+    """Synchronize torch's current stream and return (and clear) the device
+    error status (0 = OK, 6 = a bounded wait timed out)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    return int(lib().sage2_check_device_error(st))
+
+
+def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor) -> dict:
+    """Smoothing + INT4 of Q and K and the Q-smoothing correction.
+    Returns the payload dict (q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr)."""
+    B, H, N, d = _dims(q)
+    if k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must have the same shape and dtype")
+    _dims(k)
+    Np = n_pad(N)
+    NB = Np // 128
+    dev = q.device
+    out = dict(
+        q_i4=torch.empty(B, H, Np, d, dtype=torch.int8, device=dev),
+        q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
+        q_mean=torch.empty(B, H, NB, d, dtype=torch.float32, device=dev),
+        k_i4=torch.empty(B, H, Np, d, dtype=torch.int8, device=dev),
+        k_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
+        k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev),
+        qk_corr=torch.empty(B, H, NB, Np, dtype=torch.float32, device=dev),
+    )
+    st = lib().sage2_smooth_quant_qk(
+        _ptr(q), _ptr(k), _DT[q.dtype], B, H, N, d, _ptr(out["q_i4"]), _ptr(out["q_scale"]),
+        _ptr(out["q_mean"]), _ptr(out["k_i4"]), _ptr(out["k_scale"]), _ptr(out["k_mean"]),
+        _ptr(out["qk_corr"]), _stream(q))
+    _check("sage2_smooth_quant_qk", st)
+    return out
+
+
+def sage2_quant_v(v: torch.Tensor):
+    """FP8 e4m3 V per channel. Returns (v_fp8_t uint8 [B,H,d,Np], v_scale f32 [B,H,d])."""
+    B, H, N, d = _dims(v)
+    Np = n_pad(N)
+    vt = torch.empty(B, H, d, Np, dtype=torch.uint8, device=v.device)
+    vs = torch.empty(B, H, d, dtype=torch.float32, device=v.device)
+    st = lib().sage2_quant_v(_ptr(v), _DT[v.dtype], B, H, N, d, _ptr(vt), _ptr(vs), _stream(v))
+    _check("sage2_quant_v", st)
+    return vt, vs
+
+
+def sage2_attn_fwd_quantized(pay: dict, v_fp8_t: torch.Tensor, v_scale: torch.Tensor, N: int,
+                             causal: bool, sm_scale: float, out_dtype=torch.float32,
+                             out: torch.Tensor | None = None) -> torch.Tensor:
+    """The attention kernel alone, over payloads from sage2_smooth_quant_qk /
+    sage2_quant_v (or any tensors in those layouts)."""
+    B, H, Np, d = pay["q_i4"].shape
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=out_dtype, device=pay["q_i4"].device)
+    st = lib().sage2_attn_fwd_quantized(
+        _ptr(pay["q_i4"]), _ptr(pay["q_scale"]), _ptr(pay["k_i4"]), _ptr(pay["k_scale"]),
+        _ptr(pay["qk_corr"]), _ptr(v_fp8_t), _ptr(v_scale), _ptr(out), _DT[out.dtype],
+        B, H, N, d, int(bool(causal)), float(sm_scale), _stream(out))
+    _check("sage2_attn_fwd_quantized", st)
+    return out
+
+
+def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                   sm_scale: float | None = None, out_dtype=None,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """Full forward pass (quantization + correction + attention) on q's stream."""
+    B, H, N, d = _dims(q)
+    for t in (k, v):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k and v must have the same shape and dtype")
+        _dims(t)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib().sage2_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, _DT[q.dtype],
+                              _DT[out.dtype], int(bool(causal)), float(sm_scale), _stream(q))
+    _check("sage2_attn_fwd", st)
+    return out
+
+
+attn = sage2_attn_fwd
+
+
+def sage2_debug_qk_s32(q_i4: torch.Tensor, k_i4: torch.Tensor, N: int) -> torch.Tensor:
+    """Raw int32 tiles of q_i4 . k_i4^T through the tcgen05 kind::i8 path."""
+    B, H, Np, d = q_i4.shape
+    s = torch.empty(B, H, Np, Np, dtype=torch.int32, device=q_i4.device)
+    st = lib().sage2_debug_qk_s32(_ptr(q_i4), _ptr(k_i4), B, H, N, d, _ptr(s), _stream(q_i4))
+    _check("sage2_debug_qk_s32", st)
+    return s

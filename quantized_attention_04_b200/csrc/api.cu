@@ -1,0 +1,304 @@
+// C ABI of libsage2 (declared in include/sage2.h): argument validation,
+// workspace layout, tensor maps and the stream-ordered launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/sage2.h"
+#include "sage2_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace sage2 {
+
+// ------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+cudaError_t make_tmap_u8_2d(void* tmap_out, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_rows, uint32_t box_cols) {
+  auto fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};  // bytes between consecutive rows
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t elem_strides[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_cols == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUresult r = fn(reinterpret_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                        const_cast<void*>(base), dims, strides, box, elem_strides,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------ validation
+struct Dims {
+  int B, H, N, d, Np, NB;
+  int64_t BH;
+};
+
+static sage2_status check_dims(int B, int H, int N, int d, Dims* out) {
+  if (B <= 0 || H <= 0 || N <= 0) return SAGE2_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAGE2_ERR_UNSUPPORTED;
+  const int64_t BH = static_cast<int64_t>(B) * H;
+  const int64_t Np = ((static_cast<int64_t>(N) + kTile - 1) / kTile) * kTile;
+  // TMA row coordinates and grid dimensions are 32-bit; grid.y <= 65535.
+  if (BH > 65535 || BH * Np > INT32_MAX || BH * d > INT32_MAX || Np > INT32_MAX / 2)
+    return SAGE2_ERR_UNSUPPORTED;
+  out->B = B;
+  out->H = H;
+  out->N = N;
+  out->d = d;
+  out->Np = static_cast<int>(Np);
+  out->NB = static_cast<int>(Np / kTile);
+  out->BH = BH;
+  return SAGE2_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename... P>
+static sage2_status check_ptrs(P... ps) {
+  const void* arr[] = {static_cast<const void*>(ps)...};
+  for (const void* p : arr)
+    if (!p) return SAGE2_ERR_INVALID_ARG;
+  for (const void* p : arr)
+    if (!aligned16(p)) return SAGE2_ERR_MISALIGNED;
+  return SAGE2_OK;
+}
+
+static sage2_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SAGE2_OK;
+  if (e == cudaErrorMemoryAllocation) return SAGE2_ERR_NO_MEM;
+  return SAGE2_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ workspace
+struct Workspace {
+  size_t off_q_i4, off_k_i4, off_vt, off_qs, off_ks, off_qm, off_km, off_corr, off_vs, off_part,
+      off_amax, total;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static Workspace layout(const Dims& g) {
+  Workspace w{};
+  const size_t BH = static_cast<size_t>(g.BH), Np = g.Np, NB = g.NB, d = g.d;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += up256(bytes);
+    return at;
+  };
+  w.off_q_i4 = take(BH * Np * d);
+  w.off_k_i4 = take(BH * Np * d);
+  w.off_vt = take(BH * d * Np);
+  w.off_qs = take(BH * Np * 4);
+  w.off_ks = take(BH * Np * 4);
+  w.off_qm = take(BH * NB * d * 4);
+  w.off_km = take(BH * d * 4);
+  w.off_corr = take(BH * NB * Np * 4);
+  w.off_vs = take(BH * d * 4);
+  w.off_part = take(BH * NB * d * 4);
+  w.off_amax = take(BH * d * 4);
+  w.total = o;
+  return w;
+}
+
+// One stream-ordered pool per device that keeps freed memory for reuse.
+static cudaMemPool_t device_pool(int dev) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = UINT64_MAX;
+    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = p;
+  }
+  return pools[dev];
+}
+
+}  // namespace sage2
+
+using namespace sage2;
+
+extern "C" {
+
+sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int B, int H, int N,
+                                   int d, int8_t* q_i4, float* q_scale, float* q_mean,
+                                   int8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
+                                   sage2_stream_t stream) {
+  Dims g;
+  sage2_status s = check_dims(B, H, N, d, &g);
+  if (s != SAGE2_OK) return s;
+  if (dtype != SAGE2_F16 && dtype != SAGE2_BF16) return SAGE2_ERR_INVALID_ARG;
+  s = check_ptrs(q, k, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
+  if (s != SAGE2_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* part = nullptr;
+  const size_t part_bytes = static_cast<size_t>(g.BH) * g.NB * d * 4;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&part), part_bytes, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  QKArgs a{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean,
+           qk_corr, part, 0};
+  e = launch_smooth_quant_qk(a, st);
+  const cudaError_t e2 = cudaFreeAsync(part, st);
+  return from_cuda(e != cudaSuccess ? e : e2);
+}
+
+sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d, uint8_t* v_fp8_t,
+                           float* v_scale, sage2_stream_t stream) {
+  Dims g;
+  sage2_status s = check_dims(B, H, N, d, &g);
+  if (s != SAGE2_OK) return s;
+  if (dtype != SAGE2_F16 && dtype != SAGE2_BF16) return SAGE2_ERR_INVALID_ARG;
+  s = check_ptrs(v, v_fp8_t, v_scale);
+  if (s != SAGE2_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* amax = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&amax), g.BH * d * 4, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  VArgs a{v, dtype, B, H, N, d, g.Np, g.NB, v_fp8_t, v_scale, amax};
+  e = launch_quant_v(a, st);
+  const cudaError_t e2 = cudaFreeAsync(amax, st);
+  return from_cuda(e != cudaSuccess ? e : e2);
+}
+
+sage2_status sage2_attn_fwd_quantized(const int8_t* q_i4, const float* q_scale,
+                                      const int8_t* k_i4, const float* k_scale,
+                                      const float* qk_corr, const uint8_t* v_fp8_t,
+                                      const float* v_scale, void* o, int o_dtype, int B, int H,
+                                      int N, int d, int causal, float sm_scale,
+                                      sage2_stream_t stream) {
+  Dims g;
+  sage2_status s = check_dims(B, H, N, d, &g);
+  if (s != SAGE2_OK) return s;
+  if (o_dtype < SAGE2_F16 || o_dtype > SAGE2_F32) return SAGE2_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE2_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || sm_scale > 3.0e38f) return SAGE2_ERR_INVALID_ARG;
+  s = check_ptrs(q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale, o);
+  if (s != SAGE2_OK) return s;
+  AttnArgs a{q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale, o, o_dtype,
+             B,    H,       N,    d,       g.Np,    g.NB,    causal,  sm_scale};
+  return from_cuda(launch_attn(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t sage2_workspace_bytes(int B, int H, int N, int d) {
+  Dims g;
+  if (check_dims(B, H, N, d, &g) != SAGE2_OK) return 0;
+  return layout(g).total;
+}
+
+sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int N, int d, int dtype, int o_dtype, int causal, float sm_scale,
+                            sage2_stream_t stream) {
+  Dims g;
+  sage2_status s = check_dims(B, H, N, d, &g);
+  if (s != SAGE2_OK) return s;
+  if (dtype != SAGE2_F16 && dtype != SAGE2_BF16) return SAGE2_ERR_INVALID_ARG;
+  if (o_dtype < SAGE2_F16 || o_dtype > SAGE2_F32) return SAGE2_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE2_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || sm_scale > 3.0e38f) return SAGE2_ERR_INVALID_ARG;
+  s = check_ptrs(q, k, v, o);
+  if (s != SAGE2_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return SAGE2_ERR_CUDA;
+  cudaMemPool_t pool = device_pool(dev);
+  if (!pool) return SAGE2_ERR_CUDA;
+  const Workspace w = layout(g);
+  uint8_t* ws = nullptr;
+  e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), w.total, pool, st);
+  if (e != cudaSuccess) return from_cuda(e);
+
+  int8_t* q_i4 = reinterpret_cast<int8_t*>(ws + w.off_q_i4);
+  int8_t* k_i4 = reinterpret_cast<int8_t*>(ws + w.off_k_i4);
+  uint8_t* vt = ws + w.off_vt;
+  float* qs = reinterpret_cast<float*>(ws + w.off_qs);
+  float* ks = reinterpret_cast<float*>(ws + w.off_ks);
+  float* qm = reinterpret_cast<float*>(ws + w.off_qm);
+  float* km = reinterpret_cast<float*>(ws + w.off_km);
+  float* corr = reinterpret_cast<float*>(ws + w.off_corr);
+  float* vs = reinterpret_cast<float*>(ws + w.off_vs);
+  float* part = reinterpret_cast<float*>(ws + w.off_part);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
+
+  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part, causal};
+  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax};
+  AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
+              sm_scale};
+  e = launch_smooth_quant_qk(qa, st);
+  if (e == cudaSuccess) e = launch_quant_v(va, st);
+  if (e == cudaSuccess) e = launch_attn(aa, st);
+  const cudaError_t e2 = cudaFreeAsync(ws, st);
+  return from_cuda(e != cudaSuccess ? e : e2);
+}
+
+sage2_status sage2_debug_qk_s32(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int N,
+                                int d, int32_t* s_out, sage2_stream_t stream) {
+  Dims g;
+  sage2_status s = check_dims(B, H, N, d, &g);
+  if (s != SAGE2_OK) return s;
+  if (g.BH * (int64_t)g.NB * g.NB > (int64_t)INT32_MAX) return SAGE2_ERR_UNSUPPORTED;
+  if (g.BH > 65535) return SAGE2_ERR_UNSUPPORTED;
+  s = check_ptrs(q_i4, k_i4, s_out);
+  if (s != SAGE2_OK) return s;
+  return from_cuda(launch_debug_qk(q_i4, k_i4, B, H, g.Np, d, s_out,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sage2_status sage2_check_device_error(sage2_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SAGE2_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess)
+    return SAGE2_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+      return SAGE2_ERR_CUDA;
+  }
+  if (word & DEVERR_TIMEOUT) return SAGE2_ERR_TIMEOUT;
+  if (word) return SAGE2_ERR_CUDA;
+  return SAGE2_OK;
+}
+
+const char* sage2_status_string(sage2_status status) {
+  switch (status) {
+    case SAGE2_OK: return "ok";
+    case SAGE2_ERR_INVALID_ARG: return "invalid argument";
+    case SAGE2_ERR_UNSUPPORTED: return "unsupported size or head dimension";
+    case SAGE2_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case SAGE2_ERR_CUDA: return "CUDA error";
+    case SAGE2_ERR_NO_MEM: return "out of device memory";
+    case SAGE2_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int sage2_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+// Test kernel: raw s32 tiles of the INT4 product Q^ K^T through the same TMA +
+// tcgen05 kind::i8 path as the attention kernel (one 128x128 tile per CTA).
+// Lets the integer matrix product ("4-bit matrix multiplication", SageAttention2
+// abstract page, Abstract) be checked bit for bit on its own.
+#include <cuda.h>
+
+#include "sage2_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace sage2 {
+
+template <int D>
+__global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CUtensorMap tm_q,
+                                                      const __grid_constant__ CUtensorMap tm_k,
+                                                      int Np, int32_t* __restrict__ s_out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sq = base;
+  uint8_t* sk = base + 128 * D;
+  __shared__ uint64_t bar_load, bar_mma;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  const int qt = blockIdx.x, kt = blockIdx.y, bh = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_load, 1);
+    mbar_init(&bar_mma, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(&bar_load, 2 * 128 * D);
+    tma_load_2d(sq, &tm_q, &bar_load, 0, bh * Np + qt * 128);
+    tma_load_2d(sk, &tm_k, &bar_load, 0, bh * Np + kt * 128);
+    if (mbar_wait(&bar_load, 0, &abort_flag)) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_i8_s32(128, 128);
+#pragma unroll
+      for (int kk = 0; kk < D / 32; ++kk)
+        mma_i8_ss(tmem, smem_desc_kmajor(sq + 32 * kk, D), smem_desc_kmajor(sk + 32 * kk, D),
+                  idesc, kk > 0);
+      tc_commit(&bar_mma);
+    }
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bar_mma, 0, &abort_flag);
+  tc_fence_after();
+  if (ok) {
+    const int r = warp * 32 + lane;
+    int32_t* dst = s_out + (static_cast<size_t>(bh) * Np + qt * 128 + r) * Np + kt * 128;
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int u = 0; u < 32; u += 4)
+        *reinterpret_cast<int4*>(dst + c0 + u) = make_int4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+template <int D>
+static cudaError_t launch_debug_t(const int8_t* q_i4, const int8_t* k_i4, int BH, int Np,
+                                  int32_t* s_out, cudaStream_t st) {
+  alignas(64) CUtensorMap tq, tk;
+  cudaError_t e = make_tmap_u8_2d(&tq, q_i4, static_cast<uint64_t>(BH) * Np, D, 128, D);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_u8_2d(&tk, k_i4, static_cast<uint64_t>(BH) * Np, D, 128, D);
+  if (e != cudaSuccess) return e;
+  const int smem = 2 * 128 * D + 1024;
+  const int nt = Np / 128;
+  k_debug_qk_s32<D><<<dim3(nt, nt, BH), 128, smem, st>>>(tq, tk, Np, s_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_qk(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int Np, int d,
+                            int32_t* s_out, cudaStream_t st) {
+  return d == 64 ? launch_debug_t<64>(q_i4, k_i4, B * H, Np, s_out, st)
+                 : launch_debug_t<128>(q_i4, k_i4, B * H, Np, s_out, st);
+}
+
+}  // namespace sage2

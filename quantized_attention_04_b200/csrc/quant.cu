@@ -1,0 +1,349 @@
+// Smoothing and quantization kernels (HBM-bound passes).
+//
+//  k_mean_partial / k_mean_finalize : K smoothing - token mean of K per channel.
+//  k_smooth_quant                   : Q smoothing (mean of each 128-row block) and
+//                                     K smoothing applied, then INT4 per token.
+//  k_qk_corr                        : the correction qbar_blk . K_j added back
+//                                     to the INT4 product.
+//  k_v_amax / k_v_quant             : FP8 e4m3 V with one scale per channel,
+//                                     written transposed (token-contiguous).
+//
+// Method: "SageAttention2: Efficient Attention with Thorough Outlier Smoothing
+// and Per-thread INT4 Quantization" (arxiv.science abstract page, Abstract):
+// INT4 (Q,K), FP8 V, smoothing of Q; K smoothing from the title's "outlier
+// smoothing".  Every rounding below is spelled with an explicit IEEE intrinsic
+// (__fadd_rn, __fmul_rn, ...) so that no contraction or reassociation changes
+// the payload bits: the summation orders are part of the specification.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "sage2_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace sage2 {
+
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]);
+template <>
+__device__ __forceinline__ void unpack8<__half>(const uint4& u, float (&x)[8]) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void unpack8<__nv_bfloat16>(const uint4& u, float (&x)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// ---------------------------------------------------------------------------
+// K mean, pass 1: one worker (D/8 threads, 8 channels each) per 128-token
+// chunk sums its chunk token by token in ascending order (fp32).
+// grid (ceil(nchunks / workers_per_block), B*H), 256 threads.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_mean_partial(const T* __restrict__ k, int N, int nchunks,
+                                                      float* __restrict__ part) {
+  constexpr int TPR = D / 8;
+  constexpr int WPB = 256 / TPR;
+  const int bh = blockIdx.y;
+  const int worker = threadIdx.x / TPR, q8 = threadIdx.x % TPR;
+  const int chunk = blockIdx.x * WPB + worker;
+  if (chunk >= nchunks) return;
+  const int t0 = chunk * 128;
+  const int nt = min(128, N - t0);
+  const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bh * N + t0) * D) + q8;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  int t = 0;
+  for (; t + 8 <= nt; t += 8) {
+    uint4 u[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) u[s] = __ldg(src + (size_t)(t + s) * TPR);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      float x[8];
+      unpack8<T>(u[s], x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+    }
+  }
+  for (; t < nt; ++t) {
+    float x[8];
+    unpack8<T>(__ldg(src + (size_t)t * TPR), x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+  }
+  float4* dst = reinterpret_cast<float4*>(part + ((size_t)bh * nchunks + chunk) * D + q8 * 8);
+  dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// K mean, pass 2: chunk sums added in chunk order, then one fp32 division by N.
+// grid (B*H), D threads.
+__global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int N, int D,
+                                float* __restrict__ kmean) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  const float* p = part + (size_t)bh * nchunks * D + c;
+  float total = 0.f;
+  for (int ch = 0; ch < nchunks; ++ch) total = __fadd_rn(total, p[(size_t)ch * D]);
+  kmean[(size_t)bh * D + c] = __fdiv_rn(total, (float)N);
+}
+
+// ---------------------------------------------------------------------------
+// Smoothing + INT4.  grid (NB, B*H, 2): z = 0 quantizes the Q block (after
+// computing its mean), z = 1 the K block (after subtracting kbar).  256 threads.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_smooth_quant(
+    const T* __restrict__ q, const T* __restrict__ k, int N, int Np, int NB,
+    const float* __restrict__ kmean, int8_t* __restrict__ q_i4, float* __restrict__ q_scale,
+    float* __restrict__ q_mean, int8_t* __restrict__ k_i4, float* __restrict__ k_scale) {
+  __shared__ __align__(16) T tile[128][D];
+  __shared__ float mean[D];
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const bool is_q = blockIdx.z == 0;
+  const T* src = is_q ? q : k;
+  const int r0 = blk * 128;
+  const int nvalid = min(128, N - r0);
+
+  // coalesced 16-byte loads of the valid rows
+  constexpr int VPR = D / 8;  // uint4 per row
+  const uint4* g = reinterpret_cast<const uint4*>(src + ((size_t)bh * N + r0) * D);
+  uint4* s = reinterpret_cast<uint4*>(&tile[0][0]);
+  for (int i = threadIdx.x; i < nvalid * VPR; i += 256) s[i] = __ldg(g + i);
+
+  if (is_q) {
+    __syncthreads();
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      float acc = 0.f;
+      for (int r = 0; r < nvalid; ++r) acc = __fadd_rn(acc, to_f32(tile[r][c]));
+      const float m = __fdiv_rn(acc, (float)nvalid);
+      mean[c] = m;
+      q_mean[((size_t)bh * NB + blk) * D + c] = m;
+    }
+  } else {
+    if (threadIdx.x < D) mean[threadIdx.x] = kmean[(size_t)bh * D + threadIdx.x];
+  }
+  __syncthreads();
+
+  int8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * D;
+  float* scale = (is_q ? q_scale : k_scale) + (size_t)bh * Np + r0;
+  constexpr int CPL = D / 32;  // channels per lane: 4 (D=128) or 2 (D=64)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < 128; r += 8) {
+    float x[CPL];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int c = lane * CPL + i;
+      x[i] = (r < nvalid) ? __fsub_rn(to_f32(tile[r][c]), mean[c]) : 0.f;
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    uint32_t packed = 0;
+    float sc = 0.f;
+    if (amax > 0.f) {
+      sc = __fdiv_rn(amax, 7.f);
+      const float inv = __fdiv_rn(7.f, amax);
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        float v = rintf(__fmul_rn(x[i], inv));
+        v = fminf(fmaxf(v, -7.f), 7.f);
+        packed |= (static_cast<uint32_t>(static_cast<int>(v)) & 0xFFu) << (8 * i);
+      }
+    }
+    if (CPL == 4) {
+      reinterpret_cast<uint32_t*>(out + (size_t)r * D)[lane] = packed;
+    } else {
+      reinterpret_cast<uint16_t*>(out + (size_t)r * D)[lane] = static_cast<uint16_t>(packed);
+    }
+    if (lane == 0) scale[r] = sc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Q-smoothing correction C[blk][j] = sum_c qbar[blk][c] * K[j][c] (raw K), fp32
+// FMA in ascending c.  grid (Np/128, B*H), 128 threads: thread = key j.
+// first_blk_causal: when nonzero, blocks that a causal mask hides from this key
+// tile (blk < key tile) are skipped (they are never read).
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_qk_corr(const T* __restrict__ k,
+                                                 const float* __restrict__ q_mean, int N, int Np,
+                                                 int NB, int skip_masked,
+                                                 float* __restrict__ corr) {
+  __shared__ __align__(16) float qm[16][D];
+  const int kt = blockIdx.x, bh = blockIdx.y;
+  const int j = kt * 128 + threadIdx.x;
+  float kr[D];
+  if (j < N) {
+    const uint4* g = reinterpret_cast<const uint4*>(k + ((size_t)bh * N + j) * D);
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) {
+      float x[8];
+      unpack8<T>(__ldg(g + v), x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kr[v * 8 + i] = x[i];
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; ++c) kr[c] = 0.f;
+  }
+  const int b_first = skip_masked ? kt : 0;
+  for (int b0 = b_first; b0 < NB; b0 += 16) {
+    const int nb = min(16, NB - b0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb * D; i += 128)
+      (&qm[0][0])[i] = q_mean[((size_t)bh * NB + b0) * D + i];
+    __syncthreads();
+    for (int bb = 0; bb < nb; ++bb) {
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < D; c += 4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(&qm[bb][c]);
+        acc = __fmaf_rn(m4.x, kr[c], acc);
+        acc = __fmaf_rn(m4.y, kr[c + 1], acc);
+        acc = __fmaf_rn(m4.z, kr[c + 2], acc);
+        acc = __fmaf_rn(m4.w, kr[c + 3], acc);
+      }
+      corr[((size_t)bh * NB + b0 + bb) * Np + j] = acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// V, pass 1: per-channel amax over all tokens.  grid (nchunks, B*H), 256
+// threads; one 128-token chunk per block; float bits of |x| >= 0 are ordered
+// like unsigned integers, so atomicMax on the bits is exact.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
+                                                uint32_t* __restrict__ amax_bits) {
+  constexpr int TPR = D / 8;
+  constexpr int RPB = 256 / TPR;  // rows handled at once by the block
+  __shared__ float red[RPB][D];
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int r = threadIdx.x / TPR, q8 = threadIdx.x % TPR;
+  const int t0 = chunk * 128;
+  const int nt = min(128, N - t0);
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = 0.f;
+  const uint4* src = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + t0) * D) + q8;
+  for (int t = r; t < nt; t += RPB) {
+    float x[8];
+    unpack8<T>(__ldg(src + (size_t)t * TPR), x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(x[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[r][q8 * 8 + i] = m[i];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float a = 0.f;
+    for (int rr = 0; rr < RPB; ++rr) a = fmaxf(a, red[rr][threadIdx.x]);
+    atomicMax(&amax_bits[(size_t)bh * D + threadIdx.x], __float_as_uint(a));
+  }
+}
+
+// V, pass 2: codes = e4m3_rn_satfinite(V * (448/amax_c)), stored transposed.
+// grid (Np/128, B*H), 256 threads.  A warp owns one 16-token group and 32
+// consecutive channels, so its shared-memory reads are conflict-free.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N, int Np,
+                                                 const uint32_t* __restrict__ amax_bits,
+                                                 uint8_t* __restrict__ vt,
+                                                 float* __restrict__ v_scale) {
+  __shared__ __align__(16) T tile[128][D];
+  __shared__ float inv[D];
+  const int kt = blockIdx.x, bh = blockIdx.y;
+  const int t0 = kt * 128;
+  const int nvalid = max(0, min(128, N - t0));
+  constexpr int VPR = D / 8;
+  const uint4* g = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + t0) * D);
+  uint4* s = reinterpret_cast<uint4*>(&tile[0][0]);
+  for (int i = threadIdx.x; i < nvalid * VPR; i += 256) s[i] = __ldg(g + i);
+  if (threadIdx.x < D) {
+    const float a = __uint_as_float(amax_bits[(size_t)bh * D + threadIdx.x]);
+    inv[threadIdx.x] = a > 0.f ? __fdiv_rn(448.f, a) : 0.f;
+    if (kt == 0) v_scale[(size_t)bh * D + threadIdx.x] = a > 0.f ? __fdiv_rn(a, 448.f) : 0.f;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // work items: (channel group of 32, 16-token group): (D/32) * 8 items, 8 warps
+  for (int item = warp; item < (D / 32) * 8; item += 8) {
+    const int c = (item / 8) * 32 + lane;
+    const int tg = item % 8;
+    const float sc = inv[c];
+    uint32_t w[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = tg * 16 + p * 4 + h * 2;
+        const float x0 = (r < nvalid) ? __fmul_rn(to_f32(tile[r][c]), sc) : 0.f;
+        const float x1 = (r + 1 < nvalid) ? __fmul_rn(to_f32(tile[r + 1][c]), sc) : 0.f;
+        const __nv_fp8x2_storage_t two =
+            __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+        word |= static_cast<uint32_t>(two) << (16 * h);
+      }
+      w[p] = word;
+    }
+    *reinterpret_cast<uint4*>(vt + ((size_t)bh * D + c) * Np + t0 + tg * 16) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (called by the C ABI after validation).
+template <typename T, int D>
+static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
+  const int BH = a.B * a.H;
+  const int nchunks = a.NB;
+  constexpr int WPB = 256 / (D / 8);
+  k_mean_partial<T, D><<<dim3((nchunks + WPB - 1) / WPB, BH), 256, 0, st>>>(
+      static_cast<const T*>(a.k), a.N, nchunks, a.mean_part);
+  k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, nchunks, a.N, D, a.k_mean);
+  k_smooth_quant<T, D><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
+      a.q_scale, a.q_mean, a.k_i4, a.k_scale);
+  k_qk_corr<T, D><<<dim3(a.NB, BH), 128, 0, st>>>(static_cast<const T*>(a.k), a.q_mean, a.N,
+                                                  a.Np, a.NB, a.skip_masked_corr, a.qk_corr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st) {
+  if (a.dtype == 0) return a.d == 64 ? launch_qk_t<__half, 64>(a, st) : launch_qk_t<__half, 128>(a, st);
+  return a.d == 64 ? launch_qk_t<__nv_bfloat16, 64>(a, st) : launch_qk_t<__nv_bfloat16, 128>(a, st);
+}
+
+template <typename T, int D>
+static cudaError_t launch_v_t(const VArgs& a, cudaStream_t st) {
+  const int BH = a.B * a.H;
+  cudaError_t e = cudaMemsetAsync(a.amax_bits, 0, sizeof(uint32_t) * BH * D, st);
+  if (e != cudaSuccess) return e;
+  k_v_amax<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.amax_bits);
+  k_v_quant<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.Np,
+                                                  a.amax_bits, a.v_fp8_t, a.v_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st) {
+  if (a.dtype == 0) return a.d == 64 ? launch_v_t<__half, 64>(a, st) : launch_v_t<__half, 128>(a, st);
+  return a.d == 64 ? launch_v_t<__nv_bfloat16, 64>(a, st) : launch_v_t<__nv_bfloat16, 128>(a, st);
+}
+
+}  // namespace sage2

@@ -1,0 +1,63 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sage2 {
+
+constexpr int kTile = 128;  // BM = BN = 128: Q rows per block, keys per tile
+
+struct QKArgs {
+  const void* q;
+  const void* k;
+  int dtype;  // 0 fp16, 1 bf16
+  int B, H, N, d, Np, NB;
+  int8_t* q_i4;
+  float* q_scale;
+  float* q_mean;
+  int8_t* k_i4;
+  float* k_scale;
+  float* k_mean;
+  float* qk_corr;
+  float* mean_part;        // scratch [B*H, NB, d]
+  int skip_masked_corr;    // 1: skip correction blocks a causal mask hides
+};
+
+struct VArgs {
+  const void* v;
+  int dtype;
+  int B, H, N, d, Np, NB;
+  uint8_t* v_fp8_t;
+  float* v_scale;
+  uint32_t* amax_bits;     // scratch [B*H, d]
+};
+
+struct AttnArgs {
+  const int8_t* q_i4;
+  const float* q_scale;
+  const int8_t* k_i4;
+  const float* k_scale;
+  const float* qk_corr;
+  const uint8_t* v_fp8_t;
+  const float* v_scale;
+  void* o;
+  int o_dtype;  // 0 fp16, 1 bf16, 2 fp32
+  int B, H, N, d, Np, NB;
+  int causal;
+  float sm_scale;
+};
+
+cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st);
+cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_debug_qk(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int Np, int d,
+                            int32_t* s_out, cudaStream_t st);
+
+// Tensor-map creation through the driver entry point (no link-time libcuda).
+// Encodes a 2-D row-major uint8 tensor [rows, cols] with a box of
+// [box_rows, box_cols] and 128- or 64-byte swizzle (box_cols bytes).
+cudaError_t make_tmap_u8_2d(void* tmap_out, const void* base, uint64_t rows, uint64_t cols,
+                            uint32_t box_rows, uint32_t box_cols);
+
+}  // namespace sage2

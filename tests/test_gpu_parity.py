@@ -1,0 +1,162 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Payloads and integer products bit-exact; O within the
+tolerances of tests/parity.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sage2_oracle as orc
+from quantized_attention_04_b200.inputs import CONFIGS, Config, Dist, make_qkv
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qa():
+    from quantized_attention_04_b200 import build
+    build.build()
+    import quantized_attention_04_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    m.lib()
+    return m
+
+
+def small_cfg(N, d, dtype="fp16", causal=False, H=2, B=1, idx=20):
+    return Config(f"small_N{N}_d{d}", B, H, N, d, causal, dtype,
+                  q=Dist(1.0), k=Dist(3.0, outliers=2, outlier_scale=8.0), v=Dist(1.0), index=idx)
+
+
+SMALL = [
+    small_cfg(1, 64), small_cfg(17, 128, "bf16", True), small_cfg(128, 64, causal=True),
+    small_cfg(129, 128), small_cfg(300, 64, "bf16", True), small_cfg(300, 128, causal=True),
+    small_cfg(1000, 128, "bf16"), small_cfg(640, 64, causal=False, B=2, H=3),
+]
+
+
+def _cuda(cfg):
+    q, k, v = make_qkv(cfg)
+    return q, k, v, q.cuda(), k.cuda(), v.cuda()
+
+
+# ------------------------------------------------------------------ payloads
+@pytest.mark.parametrize("cfg", SMALL + [CONFIGS["C1"]], ids=lambda c: c.name)
+def test_payloads_bit_exact(qa, cfg):
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    pay = qa.sage2_smooth_quant_qk(qd, kd)
+    vt, vs = qa.sage2_quant_v(vd)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    g = {n: t.cpu().numpy() for n, t in pay.items()}
+    vt, vs = vt.cpu().numpy(), vs.cpu().numpy()
+    Np = orc.n_pad(cfg.N)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            K = P.np32(k[b, h])
+            o = orc.smooth_quant_qk(P.np32(q[b, h]), K)
+            for name in ("q_i4", "q_scale", "q_mean", "k_i4", "k_scale", "k_mean"):
+                assert P.bits_equal(g[name][b, h], o[name]), (name, b, h)
+            ovt, ovs = orc.quant_v(P.np32(v[b, h]))
+            assert P.bits_equal(vt[b, h], ovt), ("v_fp8_t", b, h)
+            assert P.bits_equal(vs[b, h], ovs), ("v_scale", b, h)
+            C = orc.qk_correction(o["q_mean"], K)
+            tol = P.corr_tolerance(o["q_mean"], K, Np, cfg.d)
+            assert (np.abs(g["qk_corr"][b, h] - C) <= tol).all(), ("qk_corr", b, h)
+
+
+# ------------------------------------------------------- integer QK^T tiles
+@pytest.mark.parametrize("cfg", [small_cfg(300, 64), small_cfg(300, 128, "bf16"),
+                                 small_cfg(129, 128, B=2, H=2)], ids=lambda c: c.name)
+def test_qk_s32_bit_exact(qa, cfg):
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    pay = qa.sage2_smooth_quant_qk(qd, kd)
+    s = qa.sage2_debug_qk_s32(pay["q_i4"], pay["k_i4"], cfg.N).cpu().numpy()
+    qi, ki = pay["q_i4"].cpu().numpy(), pay["k_i4"].cpu().numpy()
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            ref = orc.qk_int(qi[b, h], ki[b, h])
+            assert np.array_equal(s[b, h].astype(np.int64), ref), (b, h)
+
+
+def test_qk_s32_on_oracle_payloads(qa):
+    """Oracle-made INT4 values (not the GPU's) through the integer MMA path."""
+    rng = np.random.default_rng(31)
+    for d in (64, 128):
+        Np = 384
+        qi = rng.integers(-7, 8, (1, 2, Np, d)).astype(np.int8)
+        ki = rng.integers(-7, 8, (1, 2, Np, d)).astype(np.int8)
+        s = qa.sage2_debug_qk_s32(torch.from_numpy(qi).cuda(), torch.from_numpy(ki).cuda(), Np)
+        s = s.cpu().numpy()
+        for h in range(2):
+            assert np.array_equal(s[0, h].astype(np.int64), orc.qk_int(qi[0, h], ki[0, h]))
+
+
+# ------------------------------------------------------------- attention O
+@pytest.mark.parametrize("cfg", SMALL + [CONFIGS["C1"]], ids=lambda c: c.name)
+@pytest.mark.parametrize("out_dtype", [torch.float32, "input"])
+def test_attention_small_full(qa, cfg, out_dtype):
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    od = cfg.torch_dtype if out_dtype == "input" else out_dtype
+    sm = P.default_scale(cfg.d)
+    o = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out_dtype=od)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    o = P.np32(o)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
+            P.assert_o_close(o[b, h][rows], O, amb, od, (cfg.name, b, h))
+
+
+def test_attention_quantized_entry_matches_full(qa):
+    """sage2_attn_fwd_quantized over the GPU payloads gives sage2_attn_fwd's output."""
+    cfg = small_cfg(300, 128, causal=True)
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    sm = P.default_scale(cfg.d)
+    pay = qa.sage2_smooth_quant_qk(qd, kd)
+    vt, vs = qa.sage2_quant_v(vd)
+    o1 = qa.sage2_attn_fwd_quantized(pay, vt, vs, cfg.N, True, sm, torch.float32)
+    o2 = qa.sage2_attn_fwd(qd, kd, vd, causal=True, sm_scale=sm, out_dtype=torch.float32)
+    assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("name", ["C2"])
+def test_attention_config_full(qa, name):
+    cfg = CONFIGS[name]
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    sm = P.default_scale(cfg.d)
+    o = P.np32(qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm,
+                                 out_dtype=torch.float32))
+    assert qa.sage2_check_device_error() == 0
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
+            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (name, b, h))
+
+
+@pytest.mark.parametrize("name", ["C3", "C4", "C5"])
+def test_attention_config_sampled(qa, name):
+    """Full-size launch (as the bench runs it: input-dtype output); sampled
+    heads and query blocks (first, middle, last -> diagonal and ragged tails)
+    compared with the oracle; payloads of the sampled heads bit-exact."""
+    cfg = CONFIGS[name]
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    sm = P.default_scale(cfg.d)
+    o = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm)
+    pay = qa.sage2_smooth_quant_qk(qd, kd)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    nb = orc.n_pad(cfg.N) // 128
+    heads = [(0, 0), (cfg.B - 1, cfg.H - 1)]
+    blocks = sorted({0, nb // 2, nb - 1})
+    for b, h in heads:
+        opay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, q_blocks=blocks)
+        for n in ("q_i4", "q_scale", "k_i4", "k_scale", "k_mean"):
+            assert P.bits_equal(pay[n][b, h].cpu().numpy(), opay[n]), (name, n)
+        got = P.np32(o[b, h])[rows]
+        P.assert_o_close(got, O, amb, cfg.torch_dtype, (name, b, h))
+        ref = orc.attn_fp64(P.np32(q[b, h]), P.np32(k[b, h]), P.np32(v[b, h]), cfg.causal, sm,
+                            rows=rows)
+        assert abs(P.cosine(got, ref) - P.cosine(O, ref)) < 1e-4
