@@ -27,7 +27,9 @@
  *  q_i4   int8  [B,H,Np,d]   INT4 values in [-7,7] of Q - qbar_block, rows >= N are 0
  *  q_scale f32  [B,H,Np]     per-token scale amax/7 (0 for an all-zero row / pad)
  *  q_mean f32   [B,H,NB,d]   mean of each 128-row block of Q (valid rows only)
- *  k_i4   int8  [B,H,Np,d]   INT4 values of K - kbar, rows >= N are 0
+ *  k_i4   int8  [B,H,Np,d]   INT4 values of K - kbar, rows >= N are 0.  Rows are stored
+ *                            KEY-INTERLEAVED inside each 128-row block: stored row n of a
+ *                            block holds token 64*(n%2) + n/2 of that block.
  *  k_scale f32  [B,H,Np]     per-token scale
  *  k_mean f32   [B,H,d]      token mean of K
  *  qk_corr f32  [B,H,NB,Np]  q_mean[blk] . K[j] (raw K), 0 for j >= N
@@ -123,7 +125,9 @@ size_t sage2_workspace_bytes(int B, int H, int N, int d);
 /*
  * Test entry: the raw integer products S = q_i4 . k_i4^T of every 128x128
  * tile, through the same TMA + tcgen05 kind::i8 path as the attention kernel.
- *   s_out : int32 [B,H,Np,Np] (caller-allocated).
+ *   s_out : int32 [B,H,Np,Np] (caller-allocated).  Column j holds the product with
+ *           stored k_i4 row j (so, with the key-interleaved k_i4 layout, key
+ *           64*(j%2) + (j%128)/2 of block j/128).
  */
 sage2_status sage2_debug_qk_s32(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int N,
                                 int d, int32_t* s_out, sage2_stream_t stream);

@@ -7,7 +7,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/sage2.h"
+#include "sage2.h"
 #include "sage2_internal.h"
 #include "sm100_ptx.cuh"
 

@@ -5,19 +5,23 @@
 // INT4 Q^K^T product, FP8 P~ and V, and the two-level accumulation of P~V.
 //
 // One CTA = one 128-row query block of one head; 384 threads, warp-specialised:
-//   warp 0        TMA producer: Q^ tile once, then per key tile K^, V^T,
-//                 the correction chunk and the key scales (NS-stage ring).
+//   warp 0        TMA producer: the Q^ tile once, then per key tile K^, V^T,
+//                 the key scales and the correction chunk (kStages-deep ring).
 //   warp 1        MMA issuer (one thread): S = Q^ K^T with tcgen05 kind::i8
-//                 into TMEM (s32, double-buffered), then inner = P~ V~ with
-//                 kind::f8f6f4 (e4m3 x e4m3 -> f32) into a fresh TMEM
-//                 accumulator per tile (double-buffered).
+//                 into TMEM (s32, two buffers, issued two key tiles ahead), and
+//                 inner = P~ V~ with kind::f8f6f4 (e4m3 -> f32) into a fresh
+//                 TMEM accumulator per key tile (two buffers).
 //   warp 2        TMEM allocator.
-//   warps 4-7     softmax warpgroup: thread i owns query row i (TMEM lane i).
-//                 Dequantise, correct, online max/sum, exp2, P~ = e4m3(448 p)
-//                 written to shared memory in the MMA's swizzled layout.
-//   warps 8-11    correction warpgroup: outer accumulator in registers,
-//                 acc = alpha*acc + inner per tile (the second level), then
-//                 the epilogue O = acc * v_scale / l.
+//   warps 4-7,    two softmax warpgroups.  Thread (h, i) owns query row i (TMEM
+//   warps 8-11    lane i) and half h of every key tile: score columns
+//                 64h..64h+63 and output channels (d/2)h..(d/2)h+d/2-1.  Per
+//                 tile: dequantise + correct its 64 scores, publish the partial
+//                 row max, fold the previous tile's inner product into the
+//                 register accumulator (acc = alpha*acc + inner: the outer level
+//                 of the two-level accumulation) while the other half publishes,
+//                 then exp2, l, and P~ = e4m3(448 p) into shared memory (the
+//                 MMA's swizzled layout).
+// TMEM columns: S[b] at 128*b (b = 0, 1), inner[b] at 256 + d*b.
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout the kernel
 // records it in the device error word and every role leaves its loop.
 #include <cuda.h>
@@ -30,30 +34,33 @@
 
 namespace sage2 {
 
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 384;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+constexpr uint32_t kMagicBits = 0x4B400000u;     // 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;
 
 template <int D>
 struct __align__(1024) AttnSmem {
-  uint8_t q[128 * D];              // Q^ tile, K-major, swizzled (D bytes per row)
+  uint8_t q[128 * D];              // Q^ tile (K-major, swizzled)
   uint8_t k[kStages][128 * D];     // K^ tiles
   uint8_t v[kStages][D * 128];     // V^T tiles: D rows (channels) x 128 tokens
   uint8_t p[2][128 * 128];         // P~ tiles: 128 rows x 128 tokens (e4m3)
-  float corr[kStages][128];        // qk_corr[blk][tile keys]
-  float ksc[kStages][128];         // k_scale[tile keys]
-  float qsc[128];                  // q_scale[block rows]
-  float alpha[4][128];             // per-tile rescale factors, softmax -> correction
-  float lsum[128];                 // final row sums (448-scaled)
-  float vsc[D];                    // v_scale
+  // qk_corr and k_scale of the key tile: keys 0-63 at [0, 64), keys 64-127 at
+  // [68, 132).  The 16-byte gap puts the two halves (read by the two column
+  // parities of a warp in the same instruction) in different banks.
+  float corr[kStages][136];
+  float ksc[kStages][136];
+  float qsc[128];                  // q_scale of the block's rows
+  float vsc[2][D];                 // v_scale (one copy per softmax warpgroup)
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
-  uint64_t i_full[2], i_empty[2];
-  uint64_t a_full[4];
-  uint64_t l_full;
+  uint64_t s_full[2];               // S[b] written (tcgen05.commit)
+  uint64_t p_full[2];               // P~[b] written by all 8 softmax warps; this also
+                                    // says S[b] was read and inner[b] of tile t-2 folded
+  uint64_t i_full[2];               // inner[b] written (tcgen05.commit)
   uint64_t drain;
+  uint64_t offset_bar;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -63,7 +70,11 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -72,9 +83,45 @@ template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
-
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Dequantise + correct 32 scores: x' = sq_i * (sk_j * S_ij) + C_j.  The s32
+// value plus 0x4B400000, read as a float, is exactly 1.5*2^23 + S
+// (|S| <= 49*128 < 2^22); subtracting 1.5*2^23 is exact.
+__device__ __forceinline__ void dequant32(const uint32_t (&sr)[32], const float* ck,
+                                          const float* kk, float2 a2, float* x) {
+  const float2 nm2 = make_float2(-kMagic, -kMagic);
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 c4 = *reinterpret_cast<const float4*>(ck + j);
+    const float4 k4 = *reinterpret_cast<const float4*>(kk + j);
+    float2 f0 = make_float2(__uint_as_float(sr[j] + kMagicBits), __uint_as_float(sr[j + 1] + kMagicBits));
+    float2 f1 = make_float2(__uint_as_float(sr[j + 2] + kMagicBits), __uint_as_float(sr[j + 3] + kMagicBits));
+    f0 = __fadd2_rn(f0, nm2);
+    f1 = __fadd2_rn(f1, nm2);
+    f0 = __fmul2_rn(make_float2(k4.x, k4.y), f0);
+    f1 = __fmul2_rn(make_float2(k4.z, k4.w), f1);
+    f0 = __ffma2_rn(a2, f0, make_float2(c4.x, c4.y));
+    f1 = __ffma2_rn(a2, f1, make_float2(c4.z, c4.w));
+    x[j] = f0.x;
+    x[j + 1] = f0.y;
+    x[j + 2] = f1.x;
+    x[j + 3] = f1.y;
+  }
+}
+
+// acc[32 channels] = alpha * acc + inner (the outer level of the accumulation).
+__device__ __forceinline__ void fold32(float* acc, const uint32_t (&in)[32], float al) {
+  const float2 al2 = make_float2(al, al);
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const float2 r = __ffma2_rn(al2, make_float2(acc[c], acc[c + 1]),
+                                make_float2(__uint_as_float(in[c]), __uint_as_float(in[c + 1])));
+    acc[c] = r.x;
+    acc[c + 1] = r.y;
+  }
 }
 
 template <int D, int OT>
@@ -87,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int DH = D / 2;                       // output channels per softmax half
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = causal ? (NB - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
@@ -103,15 +151,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_empty[b], 4);
-      mbar_init(&sm.p_full[b], 4);
-      mbar_init(&sm.p_empty[b], 1);
+      mbar_init(&sm.p_full[b], 8);
       mbar_init(&sm.i_full[b], 1);
-      mbar_init(&sm.i_empty[b], 4);
     }
-    for (int a = 0; a < 4; ++a) mbar_init(&sm.a_full[a], 4);
-    mbar_init(&sm.l_full, 4);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.offset_bar, 4);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -123,12 +167,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tm_S = tmem;             // S[b] at columns b*128
-  const uint32_t tm_I = tmem + 256;       // inner[b] at columns 256 + b*D
 
   const int wg = warp >> 2;
   if (wg == 0) {
-    setmaxnreg_dec<56>();  // one call site for the whole warpgroup
+    setmaxnreg_dec<40>();  // one call site for the whole warpgroup
   }
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -141,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sm.q, &tm_q, &sm.q_full, 0, row0);
       bulk_load(sm.qsc, q_scale + row0, 512, &sm.q_full);
       const float* corr_row = qk_corr + (static_cast<size_t>(bh) * NB + qt) * Np;
+      const float* ks_row = k_scale + static_cast<size_t>(bh) * Np;
       int t = 0;
       for (; t < nt; ++t) {
         const int s = t % kStages;
@@ -148,8 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&sm.kv_full[s], 128 * D + D * 128 + 512 + 512);
         tma_load_2d(sm.k[s], &tm_k, &sm.kv_full[s], 0, bh * Np + t * 128);
         tma_load_2d(sm.v[s], &tm_v, &sm.kv_full[s], t * 128, bh * D);
-        bulk_load(sm.corr[s], corr_row + t * 128, 512, &sm.kv_full[s]);
-        bulk_load(sm.ksc[s], k_scale + static_cast<size_t>(bh) * Np + t * 128, 512, &sm.kv_full[s]);
+        bulk_load(sm.corr[s], corr_row + t * 128, 256, &sm.kv_full[s]);
+        bulk_load(sm.corr[s] + 68, corr_row + t * 128 + 64, 256, &sm.kv_full[s]);
+        bulk_load(sm.ksc[s], ks_row + t * 128, 256, &sm.kv_full[s]);
+        bulk_load(sm.ksc[s] + 68, ks_row + t * 128 + 64, 256, &sm.kv_full[s]);
       }
       if (*abort_flag) {
         // let the copies already issued land before the block exits
@@ -163,195 +208,226 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_i8_s32(128, 128);
       constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, D);
+      // descriptors are built once; a k-step or a stage only moves the start
+      // address field (16-byte units; shared memory is < 256 KB, no carry)
+      const uint64_t dq = smem_desc_kmajor(sm.q, D);
+      const uint64_t dk = smem_desc_kmajor(sm.k[0], D);
+      const uint64_t dv = smem_desc_kmajor(sm.v[0], 128);
+      const uint64_t dp = smem_desc_kmajor(sm.p[0], 128);
+      constexpr uint32_t kStageK = (128 * D) >> 4, kStageV = (D * 128) >> 4, kStageP = (128 * 128) >> 4;
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
-      auto issue_pv = [&](int u) -> bool {
+      auto issue_qk = [&](int u) -> bool {
         const int s = u % kStages, b = u & 1;
-        if (!mbar_wait(&sm.p_full[b], (u >> 1) & 1, abort_flag)) return false;
-        if (u >= 2 && !mbar_wait(&sm.i_empty[b], ((u >> 1) - 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&sm.kv_full[s], (u / kStages) & 1, abort_flag)) return false;
+        // S[b] is free once the softmax of tile u-2 is past its P~ store
+        if (u >= 2 && !mbar_wait(&sm.p_full[b], ((u >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        const uint64_t kb = dk + s * kStageK;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_f8_ss(tm_I + b * D, smem_desc_kmajor(sm.p[b] + 32 * kk, 128),
-                    smem_desc_kmajor(sm.v[s] + 32 * kk, 128), idesc_pv, kk > 0);
-        }
-        tc_commit(&sm.i_full[b]);
-        tc_commit(&sm.kv_empty[s]);
-        tc_commit(&sm.p_empty[b]);
+        for (int kk = 0; kk < D / 32; ++kk) mma_i8_ss(tmem + b * 128, dq + 2 * kk, kb + 2 * kk, idesc_qk, kk > 0);
+        tc_commit(&sm.s_full[b]);
         return true;
       };
-      for (int t = 0; ok && t < nt; ++t) {
-        const int s = t % kStages, b = t & 1;
-        if (!mbar_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; break; }
-        if (t >= 2 && !mbar_wait(&sm.s_empty[b], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      auto issue_pv = [&](int u) -> bool {
+        const int s = u % kStages, b = u & 1;
+        // P~(u) is written; inner[b] was folded (tile u-2) before that arrive
+        if (!mbar_wait(&sm.p_full[b], (u >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        const uint64_t pb = dp + b * kStageP, vb = dv + s * kStageV;
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk) {
-          mma_i8_ss(tm_S + b * 128, smem_desc_kmajor(sm.q + 32 * kk, D),
-                    smem_desc_kmajor(sm.k[s] + 32 * kk, D), idesc_qk, kk > 0);
-        }
-        tc_commit(&sm.s_full[b]);
-        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + 256 + b * D, pb + 2 * kk, vb + 2 * kk, idesc_pv, kk > 0);
+        tc_commit(&sm.i_full[b]);
+        tc_commit(&sm.kv_empty[s]);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && nt > 1) ok = issue_qk(1);
+      for (int t = 0; ok && t < nt; ++t) {
+        // both wait for the end of the softmax of tile t; PV first, its result
+        // is needed one tile earlier than S(t+2)
+        if (!issue_pv(t)) { ok = false; break; }
+        if (t + 2 < nt && !issue_qk(t + 2)) { ok = false; break; }
       }
-      if (ok) ok = issue_pv(nt - 1);
       if (!ok) {
         // wait for every MMA issued so far before the block frees TMEM
         tc_commit(&sm.drain);
         mbar_wait(&sm.drain, 0, nullptr);
       }
     }
-  } else if (wg == 0) {
-    // warps 2 and 3: nothing until the final barrier
-  } else if (wg == 1) {
-    // ------------------------------------------------------------ softmax
-    setmaxnreg_inc<216>();
-    const int r = (warp - 4) * 32 + lane;                 // query row in the block
-    const int row = qt * 128 + r;                         // query row in the head
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
-    float m = -INFINITY, l = 0.f;
-    bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
+  } else if (wg >= 1) {
+    // ------------------------------------------------------------ softmax warpgroups
+    // Raised inside the branch it governs, so that the compiler allocates this
+    // role's code against the larger budget (40*128 + 232*256 <= 168*384).
+    setmaxnreg_inc<232>();
+    // The .16x64b TMEM loads give thread t of a warp lane (t>>2) + 8*(t&1) of
+    // a 16-lane group and every other column, parity (t>>1)&1.  Warpgroup h
+    // takes lanes 16h..16h+15 of each 32-lane quadrant, so every query row is
+    // owned by the two threads t and t^2 of one warp.  With the key-interleaved
+    // K^ layout, the score columns of parity `par` are the 64 consecutive keys
+    // 64*par .. 64*par+63 of the tile, and the inner-product columns of parity
+    // `par` are the output channels 2k + par.
+    const int h = wg - 1;
+    const int quad = warp & 3;
+    const int par = (lane >> 1) & 1;
+    const int r = 32 * quad + 16 * h + (lane >> 2) + 8 * (lane & 1);   // row in the block
+    const int row = qt * 128 + r;                                       // row in the head
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * quad + 16 * h) << 16;
+    const uint32_t tS = tmem + lane_addr;                 // + 128*b: S buffer b
+    const uint32_t tI = tmem + lane_addr + 256;           // + D*b: inner buffer b
+    for (int i = threadIdx.x - 128 * wg; i < D; i += 128)
+      sm.vsc[h][i] = v_scale[static_cast<size_t>(bh) * D + i];
+    named_bar_sync(1 + h, 128);
+    float acc[DH];                                        // channels 2k + par
+#pragma unroll
+    for (int c = 0; c < DH; ++c) acc[c] = 0.f;
+    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag);
     const float a = ok ? sm.qsc[r] : 0.f;
+    const float2 a2 = make_float2(a, a);
+    const float2 L2 = make_float2(L, L);
+    // the second warpgroup starts half a tile late, so that one group's exp2
+    // phase overlaps the other group's dequantisation
+    if (ok && h == 1) ok = mbar_wait_warp(&sm.offset_bar, 0, abort_flag);
+
     for (int t = 0; ok && t < nt; ++t) {
       const int s = t % kStages, b = t & 1;
-      if (!mbar_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&sm.s_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&sm.s_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tm_S + b * 128 + lane_off + 0, s0);
-      tmem_ld32(tm_S + b * 128 + lane_off + 32, s1);
-      tmem_ld32(tm_S + b * 128 + lane_off + 64, s2);
-      tmem_ld32(tm_S + b * 128 + lane_off + 96, s3);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_empty[b]);
-
-      // x' = sq_i * (sk_j * S_ij) + C_j   (natural units; L applied in exp2)
-      float x[128];
-      const float* ck = sm.corr[s];
-      const float* kk = sm.ksc[s];
+      float x[64];                                        // keys 64*par + k
+      {
+        uint32_t s0[32], s1[32];
+        tmem_ld16x64_32(tS + b * 128, s0);
+        tmem_ld16x64_32(tS + b * 128 + 64, s1);
+        tmem_ld_wait();
+        if (!mbar_wait_warp(&sm.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; break; }
+        dequant32(s0, sm.corr[s] + 68 * par, sm.ksc[s] + 68 * par, a2, x);
+        dequant32(s1, sm.corr[s] + 68 * par + 32, sm.ksc[s] + 68 * par + 32, a2, x + 32);
+      }
+      if ((causal && t == qt) || (tail && t == NB - 1)) {
 #pragma unroll
-      for (int j = 0; j < 128; j += 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(ck + j);
-        const float4 k4 = *reinterpret_cast<const float4*>(kk + j);
-        const float cj[4] = {c4.x, c4.y, c4.z, c4.w};
-        const float kj[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          // exact int -> float: |S| <= 49*128 < 2^22
-          const uint32_t sv = (j < 32) ? s0[j + u] : (j < 64) ? s1[j - 32 + u]
-                            : (j < 96) ? s2[j - 64 + u] : s3[j - 96 + u];
-          const float sf = __int_as_float(static_cast<int>(sv) + 0x4B400000) - 12582912.f;
-          x[j + u] = fmaf(a, kj[u] * sf, cj[u]);
+        for (int k = 0; k < 64; ++k) {
+          const int key = t * 128 + 64 * par + k;
+          if (key >= N || (causal && key > row)) x[k] = -INFINITY;
         }
       }
-      const bool need_mask = (causal && t == qt) || (tail && t == NB - 1);
-      if (need_mask) {
+      float mx8[8];
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          const int key = t * 128 + j;
-          if (key >= N || (causal && key > row)) x[j] = -INFINITY;
-        }
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int j = 1; j < 128; ++j) mx = fmaxf(mx, x[j]);
+      for (int g = 0; g < 8; ++g)
+        mx8[g] = max3f(max3f(x[8 * g], x[8 * g + 1], x[8 * g + 2]),
+                       max3f(x[8 * g + 3], x[8 * g + 4], x[8 * g + 5]),
+                       fmaxf(x[8 * g + 6], x[8 * g + 7]));
+      float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                       fmaxf(mx8[6], mx8[7]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));   // the row's other half
+      if (h == 0 && t == 0) { __syncwarp(); if (lane == 0) mbar_arrive(&sm.offset_bar); }
       const float m_new = fmaxf(m, mx);
       const float alpha = ex2((m - m_new) * L);           // 0 on the first tile
       const float base = m_new * L - kLog2_448;           // p448 = 448 * exp2((x'-m)L)
-      // the P~ buffer of this parity is free once the PV product of tile t-2 is done
-      if (t >= 2 && !mbar_wait(&sm.p_empty[b], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-      // row r of the P~ tile: 8 chunks of 16 bytes, chunk index xor (r & 7)
+      const float2 nb2 = make_float2(-base, -base);
+      // the P~ buffer of this parity is free: PV(t-2) completed before i_full of
+      // tile t-2 fired, which this thread waited for in the previous tile
       uint8_t* prow = sm.p[b] + r * 128;
-      float sum = 0.f;
+      float2 sumA = make_float2(0.f, 0.f), sumB = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int j = c * 16 + u * 4;
-          const float p0 = ex2(fmaf(x[j + 0], L, -base));
-          const float p1 = ex2(fmaf(x[j + 1], L, -base));
-          const float p2 = ex2(fmaf(x[j + 2], L, -base));
-          const float p3 = ex2(fmaf(x[j + 3], L, -base));
-          sum += (p0 + p1) + (p2 + p3);
-          const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
-          const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
+          float2 e0 = __ffma2_rn(make_float2(x[j], x[j + 1]), L2, nb2);
+          float2 e1 = __ffma2_rn(make_float2(x[j + 2], x[j + 3]), L2, nb2);
+          e0.x = ex2(e0.x);
+          e0.y = ex2(e0.y);
+          e1.x = ex2(e1.x);
+          e1.y = ex2(e1.y);
+          sumA = __fadd2_rn(sumA, e0);
+          sumB = __fadd2_rn(sumB, e1);
+          const uint32_t lo = __nv_cvt_float2_to_fp8x2(e0, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t hi = __nv_cvt_float2_to_fp8x2(e1, __NV_SATFINITE, __NV_E4M3);
           w[u] = lo | (hi << 16);
         }
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        const int chunk = 4 * par + c;                    // 16-byte chunk of the 128-byte row
+        *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      l = alpha * l + sum;
-      m = m_new;
       fence_proxy_async_smem();
-      sm.alpha[t & 3][r] = alpha;
+      tc_fence_before();                                  // S(t) and inner(t-2) reads are done
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.p_full[b]);
-        mbar_arrive(&sm.a_full[t & 3]);
-      }
-    }
-    sm.lsum[r] = l;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.l_full);
-  } else {
-    // ------------------------------------------------------------ correction
-    setmaxnreg_inc<216>();
-    const int r = (warp - 8) * 32 + lane;
-    const int row = qt * 128 + r;
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 8) * 32) << 16;
-    if (r < D) sm.vsc[r] = v_scale[static_cast<size_t>(bh) * D + r];
-    named_bar_sync(1, 128);
-    float acc[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) acc[c] = 0.f;
-    bool ok = true;
-    for (int t = 0; ok && t < nt; ++t) {
-      const int b = t & 1;
-      if (!mbar_wait(&sm.i_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&sm.a_full[t & 3], (t >> 2) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const float al = sm.alpha[t & 3][r];
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tm_I + b * D + lane_off + c0, v);
+      if (lane == 0) mbar_arrive(&sm.p_full[b]);
+      const float2 sum2 = __fadd2_rn(sumA, sumB);
+      l = alpha * l + (sum2.x + sum2.y);
+      m = m_new;
+
+      // outer level for the previous tile, whose PV product ran meanwhile
+      if (t >= 1) {
+        const int u = t - 1, ub = u & 1;
+        if (!mbar_wait_warp(&sm.i_full[ub], (u >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t in0[32], in1[32];
+        tmem_ld16x64_32(tI + ub * D, in0);
+        if (DH == 64) tmem_ld16x64_32(tI + ub * D + 64, in1);
         tmem_ld_wait();
-#pragma unroll
-        for (int u = 0; u < 32; ++u) acc[c0 + u] = fmaf(al, acc[c0 + u], __uint_as_float(v[u]));
+        fold32(acc, in0, alpha_prev);
+        if (DH == 64) fold32(acc + (DH == 64 ? 32 : 0), in1, alpha_prev);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.i_empty[b]);
+      alpha_prev = alpha;
     }
-    if (ok && mbar_wait(&sm.l_full, 0, abort_flag) && row < N) {
-      const float inv_l = 1.0f / sm.lsum[r];
-      const size_t obase = (static_cast<size_t>(bh) * N + row) * D;
-      if (OT == 2) {
-        float* o = static_cast<float*>(out) + obase;
+    if (ok) {
+      const int u = nt - 1, ub = u & 1;
+      ok = mbar_wait_warp(&sm.i_full[ub], (u >> 1) & 1, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        uint32_t in0[32], in1[32];
+        tmem_ld16x64_32(tI + ub * D, in0);
+        if (DH == 64) tmem_ld16x64_32(tI + ub * D + 64, in1);
+        tmem_ld_wait();
+        fold32(acc, in0, alpha_prev);
+        if (DH == 64) fold32(acc + (DH == 64 ? 32 : 0), in1, alpha_prev);
+      }
+    }
+    if (ok) {
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const float inv_l = 1.0f / l;
+      // swap half of the channels with the row's other thread so that each
+      // thread holds D/2 consecutive output channels: (D/2)*par + i
+      float o[DH];
 #pragma unroll
-        for (int c = 0; c < D; c += 4) {
-          *reinterpret_cast<float4*>(o + c) =
-              make_float4(acc[c] * sm.vsc[c] * inv_l, acc[c + 1] * sm.vsc[c + 1] * inv_l,
-                          acc[c + 2] * sm.vsc[c + 2] * inv_l, acc[c + 3] * sm.vsc[c + 3] * inv_l);
-        }
-      } else {
-        uint16_t* o = static_cast<uint16_t*>(out) + obase;
+      for (int i = 0; i < DH / 2; ++i) {
+        const float send = par ? acc[i] : acc[DH / 2 + i];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+        const float own = par ? acc[DH / 2 + i] : acc[i];
+        o[2 * i] = par ? recv : own;
+        o[2 * i + 1] = par ? own : recv;
+      }
+      if (row < N) {
+        const float* vs = sm.vsc[h] + DH * par;
+        const size_t obase = (static_cast<size_t>(bh) * N + row) * D + DH * par;
+        if (OT == 2) {
+          float* op = static_cast<float*>(out) + obase;
 #pragma unroll
-        for (int c = 0; c < D; c += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float f0 = acc[c + 2 * u] * sm.vsc[c + 2 * u] * inv_l;
-            const float f1 = acc[c + 2 * u + 1] * sm.vsc[c + 2 * u + 1] * inv_l;
-            if (OT == 0) {
-              const __half2 h = __floats2half2_rn(f0, f1);
-              w[u] = *reinterpret_cast<const uint32_t*>(&h);
-            } else {
-              const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
-              w[u] = *reinterpret_cast<const uint32_t*>(&h);
-            }
+          for (int c = 0; c < DH; c += 4) {
+            *reinterpret_cast<float4*>(op + c) =
+                make_float4(o[c] * vs[c] * inv_l, o[c + 1] * vs[c + 1] * inv_l,
+                            o[c + 2] * vs[c + 2] * inv_l, o[c + 3] * vs[c + 3] * inv_l);
           }
-          *reinterpret_cast<uint4*>(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+          uint16_t* op = static_cast<uint16_t*>(out) + obase;
+#pragma unroll
+          for (int c = 0; c < DH; c += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float f0 = o[c + 2 * u] * vs[c + 2 * u] * inv_l;
+              const float f1 = o[c + 2 * u + 1] * vs[c + 2 * u + 1] * inv_l;
+              if (OT == 0) {
+                const __half2 hv = __floats2half2_rn(f0, f1);
+                w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+              } else {
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(f0, f1);
+                w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+            }
+            *reinterpret_cast<uint4*>(op + c) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
     }

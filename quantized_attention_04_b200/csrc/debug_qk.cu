@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
     }
   }
   __syncwarp();
-  const bool ok = mbar_wait(&bar_mma, 0, &abort_flag);
+  const bool ok = mbar_wait_warp(&bar_mma, 0, &abort_flag);
   tc_fence_after();
   if (ok) {
     const int r = warp * 32 + lane;

@@ -141,6 +141,10 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
 
   int8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * D;
   float* scale = (is_q ? q_scale : k_scale) + (size_t)bh * Np + r0;
+  // K^ rows are stored key-interleaved inside each 128-row block: token j of
+  // the block goes to stored row 2*(j % 64) + j / 64, so that stored row n
+  // holds token 64*(n % 2) + n / 2 (the attention kernel's TMEM loads then give
+  // each thread 64 consecutive keys).  Q^ rows keep their natural order.
   constexpr int CPL = D / 32;  // channels per lane: 4 (D=128) or 2 (D=64)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int r = warp; r < 128; r += 8) {
@@ -166,10 +170,11 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
         packed |= (static_cast<uint32_t>(static_cast<int>(v)) & 0xFFu) << (8 * i);
       }
     }
+    const int srow = is_q ? r : 2 * (r & 63) + (r >> 6);
     if (CPL == 4) {
-      reinterpret_cast<uint32_t*>(out + (size_t)r * D)[lane] = packed;
+      reinterpret_cast<uint32_t*>(out + (size_t)srow * D)[lane] = packed;
     } else {
-      reinterpret_cast<uint16_t*>(out + (size_t)r * D)[lane] = static_cast<uint16_t>(packed);
+      reinterpret_cast<uint16_t*>(out + (size_t)srow * D)[lane] = static_cast<uint16_t>(packed);
     }
     if (lane == 0) scale[r] = sc;
   }

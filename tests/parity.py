@@ -78,5 +78,14 @@ def bits_equal(a: np.ndarray, b: np.ndarray) -> bool:
     return np.array_equal(a, b)
 
 
+def key_interleave(Np: int) -> np.ndarray:
+    """Index map of the library's key-interleaved k_i4 row order: stored row n
+    of each 128-row block holds token 64*(n % 2) + n // 2 of that block, so
+    stored = natural[key_interleave(Np)]."""
+    n = np.arange(Np)
+    blk, j = n // 128, n % 128
+    return blk * 128 + 64 * (j % 2) + j // 2
+
+
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)

@@ -56,6 +56,7 @@ def test_payloads_bit_exact(qa, cfg):
         for h in range(cfg.H):
             K = P.np32(k[b, h])
             o = orc.smooth_quant_qk(P.np32(q[b, h]), K)
+            o["k_i4"] = o["k_i4"][P.key_interleave(Np)]       # the library's row order
             for name in ("q_i4", "q_scale", "q_mean", "k_i4", "k_scale", "k_mean"):
                 assert P.bits_equal(g[name][b, h], o[name]), (name, b, h)
             ovt, ovs = orc.quant_v(P.np32(v[b, h]))
@@ -76,8 +77,13 @@ def test_qk_s32_bit_exact(qa, cfg):
     qi, ki = pay["q_i4"].cpu().numpy(), pay["k_i4"].cpu().numpy()
     for b in range(cfg.B):
         for h in range(cfg.H):
-            ref = orc.qk_int(qi[b, h], ki[b, h])
+            ref = orc.qk_int(qi[b, h], ki[b, h])        # columns follow the stored k_i4 rows
             assert np.array_equal(s[b, h].astype(np.int64), ref), (b, h)
+            # and, through the documented row order, the oracle's own K^ in token order
+            Q = P.np32(q[b, h]); K = P.np32(k[b, h])
+            o = orc.smooth_quant_qk(Q, K)
+            ref2 = orc.qk_int(o["q_i4"], o["k_i4"])[:, P.key_interleave(qi.shape[2])]
+            assert np.array_equal(s[b, h].astype(np.int64), ref2), (b, h)
 
 
 def test_qk_s32_on_oracle_payloads(qa):
@@ -153,6 +159,7 @@ def test_attention_config_sampled(qa, name):
     blocks = sorted({0, nb // 2, nb - 1})
     for b, h in heads:
         opay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, q_blocks=blocks)
+        opay["k_i4"] = opay["k_i4"][P.key_interleave(opay["k_i4"].shape[0])]
         for n in ("q_i4", "q_scale", "k_i4", "k_scale", "k_mean"):
             assert P.bits_equal(pay[n][b, h].cpu().numpy(), opay[n]), (name, n)
         got = P.np32(o[b, h])[rows]
