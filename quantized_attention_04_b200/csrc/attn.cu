@@ -55,7 +55,9 @@ struct __align__(1024) AttnSmem {
   float vsc[2][D];                 // v_scale (one copy per softmax warpgroup)
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2];               // S[b] written (tcgen05.commit)
+  uint64_t s_full[2];               // two arrivals: the MMA thread once it saw the key
+                                    // tile land (so its scales are visible to whoever
+                                    // acquires this barrier), and the commit of S[b]
   uint64_t p_full[2];               // P~[b] written by all 8 softmax warps; this also
                                     // says S[b] was read and inner[b] of tile t-2 folded
   uint64_t i_full[2];               // inner[b] written (tcgen05.commit)
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_full[b], 2);
       mbar_init(&sm.p_full[b], 8);
       mbar_init(&sm.i_full[b], 1);
     }
@@ -221,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&sm.kv_full[s], (u / kStages) & 1, abort_flag)) return false;
         // S[b] is free once the softmax of tile u-2 is past its P~ store
         if (u >= 2 && !mbar_wait(&sm.p_full[b], ((u >> 1) - 1) & 1, abort_flag)) return false;
+        mbar_arrive(&sm.s_full[b]);                       // releases the kv_full acquire
         tc_fence_after();
         const uint64_t kb = dk + s * kStageK;
 #pragma unroll
@@ -299,7 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16x64_32(tS + b * 128, s0);
         tmem_ld16x64_32(tS + b * 128 + 64, s1);
         tmem_ld_wait();
-        if (!mbar_wait_warp(&sm.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; break; }
+        // the key scales and correction chunk of stage s are visible: s_full
+        // also carries the MMA thread's release after it acquired kv_full
         dequant32(s0, sm.corr[s] + 68 * par, sm.ksc[s] + 68 * par, a2, x);
         dequant32(s1, sm.corr[s] + 68 * par + 32, sm.ksc[s] + 68 * par + 32, a2, x + 32);
       }
