@@ -56,7 +56,8 @@ typedef enum {
   SAGE2_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned              */
   SAGE2_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed   */
   SAGE2_ERR_NO_MEM = 5,      /* workspace allocation failed                   */
-  SAGE2_ERR_TIMEOUT = 6      /* a kernel's bounded wait ran out (device word) */
+  SAGE2_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (device word) */
+  SAGE2_ERR_TOO_LARGE = 7    /* scratch needed exceeds the fixed no-allocation buffer */
 } sage2_status;
 
 typedef enum { SAGE2_F16 = 0, SAGE2_BF16 = 1, SAGE2_F32 = 2 } sage2_dtype;
@@ -118,6 +119,25 @@ sage2_status sage2_attn_fwd_quantized(const int8_t* q_i4, const float* q_scale,
 sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
                             int N, int d, int dtype, int o_dtype, int causal, float sm_scale,
                             sage2_stream_t stream);
+
+/*
+ * The same forward pass as sage2_attn_fwd, for callers that must not have the
+ * library allocate device memory while they run (hosts that forbid allocator
+ * calls after start-up, frameworks that account for every device byte
+ * themselves).  The paper has no counterpart: this is a deployment variant.
+ * Scratch comes from one fixed 64 MiB device array that every GPU loading the
+ * library holds until exit; no cudaMalloc/cudaFree/pool call is made.
+ *   - Problems with sage2_workspace_bytes() > 64 MiB return SAGE2_ERR_TOO_LARGE
+ *     before any launch.
+ *   - The first call on a device looks the array's address up
+ *     (cudaGetSymbolAddress) and caches it: make it before any stream capture.
+ *   - All calls share the array; each clears what must start at zero.  Calls
+ *     whose GPU work overlaps race on it: order them on one stream.
+ * Arguments, layouts and other statuses as sage2_attn_fwd.
+ */
+sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B,
+                                    int H, int N, int d, int dtype, int o_dtype, int causal,
+                                    float sm_scale, sage2_stream_t stream);
 
 /* Bytes of workspace sage2_attn_fwd takes for this problem (0 on bad sizes). */
 size_t sage2_workspace_bytes(int B, int H, int N, int d);

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "sage2_smooth_quant_qk", "sage2_quant_v", "sage2_attn_fwd_quantized", "sage2_attn_fwd",
-    "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
+    "sage2_attn_fwd_noalloc", "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
     "sage2_status_string", "sage2_version", "attn", "Sage2Error", "lib", "LIB_PATH",
 ]
 
@@ -28,7 +28,7 @@ F16, BF16, F32 = 0, 1, 2
 _DT = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
 STATUS = {0: "SAGE2_OK", 1: "SAGE2_ERR_INVALID_ARG", 2: "SAGE2_ERR_UNSUPPORTED",
           3: "SAGE2_ERR_MISALIGNED", 4: "SAGE2_ERR_CUDA", 5: "SAGE2_ERR_NO_MEM",
-          6: "SAGE2_ERR_TIMEOUT"}
+          6: "SAGE2_ERR_TIMEOUT", 7: "SAGE2_ERR_TOO_LARGE"}
 
 _lib = None
 _P = ctypes.c_void_p
@@ -39,6 +39,7 @@ _SIGS = {
     "sage2_quant_v": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sage2_attn_fwd_quantized": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage2_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sage2_attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage2_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "sage2_debug_qk_s32": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "sage2_check_device_error": (_I, [_P]),
@@ -191,6 +192,27 @@ def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bo
 
 
 attn = sage2_attn_fwd
+
+
+def sage2_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                           sm_scale: float | None = None, out_dtype=None,
+                           out: torch.Tensor | None = None) -> torch.Tensor:
+    """sage2_attn_fwd without any device allocation by the library: the scratch
+    is the library's fixed 64 MiB device array (see include/sage2.h)."""
+    B, H, N, d = _dims(q)
+    for t in (k, v):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k and v must have the same shape and dtype")
+        _dims(t)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib().sage2_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
+                                      _DT[q.dtype], _DT[out.dtype], int(bool(causal)),
+                                      float(sm_scale), _stream(q))
+    _check("sage2_attn_fwd_noalloc", st)
+    return out
 
 
 def sage2_debug_qk_s32(q_i4: torch.Tensor, k_i4: torch.Tensor, N: int) -> torch.Tensor:

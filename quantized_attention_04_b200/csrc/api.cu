@@ -295,6 +295,7 @@ const char* sage2_status_string(sage2_status status) {
     case SAGE2_ERR_CUDA: return "CUDA error";
     case SAGE2_ERR_NO_MEM: return "out of device memory";
     case SAGE2_ERR_TIMEOUT: return "device wait timed out";
+    case SAGE2_ERR_TOO_LARGE: return "scratch needed exceeds the fixed no-allocation buffer";
   }
   return "unknown status";
 }

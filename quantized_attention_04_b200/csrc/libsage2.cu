@@ -5,3 +5,4 @@
 #include "debug_qk.cu"
 #include "attn.cu"
 #include "api.cu"
+#include "noalloc.cu"
