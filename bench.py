@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 from quantized_attention_04_b200.inputs import CONFIGS, make_qkv  # noqa: E402
 
 METRIC = "quantized attention TOPS (4*B*H*N^2*d/t, halved if causal)"
-KERNELS_PER_STEP = 7   # k_mean_partial, k_mean_finalize, k_smooth_quant, k_qk_corr,
+KERNELS_PER_STEP = 8   # k_mean_partial, k_mean_finalize, k_smooth_quant, k_qbar_split, k_qk_corr_tc,
                        # k_v_amax, k_v_quant, k_attn_fwd
 
 

@@ -46,6 +46,31 @@ cudaError_t make_tmap_u8_2d(void* tmap_out, const void* base, uint64_t rows, uin
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_tmap(void* tmap_out, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, int elem_bytes,
+                      int swizzle_bytes) {
+  auto fn = get_encode_fn();
+  if (!fn || rank < 1 || rank > 5) return cudaErrorNotSupported;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+  const CUtensorMapDataType ty = elem_bytes == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUresult r = fn(reinterpret_cast<CUtensorMap*>(tmap_out), ty, rank, const_cast<void*>(base),
+                        d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // ------------------------------------------------------------ validation
 struct Dims {
   int B, H, N, d, Np, NB;
@@ -91,7 +116,7 @@ static sage2_status from_cuda(cudaError_t e) {
 // ------------------------------------------------------------ workspace
 struct Workspace {
   size_t off_q_i4, off_k_i4, off_vt, off_qs, off_ks, off_qm, off_km, off_corr, off_vs, off_part,
-      off_amax, total;
+      off_amax, off_qsplit, total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -116,6 +141,7 @@ static Workspace layout(const Dims& g) {
   w.off_vs = take(BH * d * 4);
   w.off_part = take(BH * NB * d * 4);
   w.off_amax = take(BH * d * 4);
+  w.off_qsplit = take(3 * BH * ((NB + 127) / 128) * 128 * d * 2);
   w.total = o;
   return w;
 }
@@ -157,14 +183,22 @@ sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int 
   s = check_ptrs(q, k, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
   if (s != SAGE2_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* part = nullptr;
-  const size_t part_bytes = static_cast<size_t>(g.BH) * g.NB * d * 4;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&part), part_bytes, st);
+  // scratch: the K-mean partial sums and the split q_mean terms
+  const size_t part_bytes = up256(static_cast<size_t>(g.BH) * g.NB * d * 4);
+  const size_t split_bytes =
+      up256(3 * static_cast<size_t>(g.BH) * ((g.NB + 127) / 128) * 128 * d * 2);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE2_ERR_CUDA;
+  cudaMemPool_t pool = device_pool(dev);
+  if (!pool) return SAGE2_ERR_CUDA;
+  uint8_t* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch),
+                                          part_bytes + split_bytes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
   QKArgs a{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean,
-           qk_corr, part, 0};
+           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, 0};
   e = launch_smooth_quant_qk(a, st);
-  const cudaError_t e2 = cudaFreeAsync(part, st);
+  const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
 }
 
@@ -246,7 +280,8 @@ sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o
   float* part = reinterpret_cast<float*>(ws + w.off_part);
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
 
-  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part, causal};
+  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
+            ws + w.off_qsplit, causal};
   VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax};
   AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
               sm_scale};

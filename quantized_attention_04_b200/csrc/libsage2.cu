@@ -2,6 +2,7 @@
 // (sage2::g_device_error), which whole-program CUDA compilation only allows
 // inside one translation unit.
 #include "quant.cu"
+#include "corr.cu"
 #include "debug_qk.cu"
 #include "attn.cu"
 #include "api.cu"

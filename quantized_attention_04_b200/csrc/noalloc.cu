@@ -98,7 +98,8 @@ extern "C" sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, con
   float* part = reinterpret_cast<float*>(ws + w.off_part);
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
 
-  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part, causal};
+  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
+            ws + w.off_qsplit, causal};
   VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax};  // amax is cleared on the stream
   AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
               sm_scale};

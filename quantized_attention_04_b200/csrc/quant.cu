@@ -3,8 +3,7 @@
 //  k_mean_partial / k_mean_finalize : K smoothing - token mean of K per channel.
 //  k_smooth_quant                   : Q smoothing (mean of each 128-row block) and
 //                                     K smoothing applied, then INT4 per token.
-//  k_qk_corr                        : the correction qbar_blk . K_j added back
-//                                     to the INT4 product.
+//  (the correction qbar_blk . K_j added back to the INT4 product is in corr.cu)
 //  k_v_amax / k_v_quant             : FP8 e4m3 V with one scale per channel,
 //                                     written transposed (token-contiguous).
 //
@@ -181,55 +180,6 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
 }
 
 // ---------------------------------------------------------------------------
-// Q-smoothing correction C[blk][j] = sum_c qbar[blk][c] * K[j][c] (raw K), fp32
-// FMA in ascending c.  grid (Np/128, B*H), 128 threads: thread = key j.
-// first_blk_causal: when nonzero, blocks that a causal mask hides from this key
-// tile (blk < key tile) are skipped (they are never read).
-template <typename T, int D>
-__global__ void __launch_bounds__(128) k_qk_corr(const T* __restrict__ k,
-                                                 const float* __restrict__ q_mean, int N, int Np,
-                                                 int NB, int skip_masked,
-                                                 float* __restrict__ corr) {
-  __shared__ __align__(16) float qm[16][D];
-  const int kt = blockIdx.x, bh = blockIdx.y;
-  const int j = kt * 128 + threadIdx.x;
-  float kr[D];
-  if (j < N) {
-    const uint4* g = reinterpret_cast<const uint4*>(k + ((size_t)bh * N + j) * D);
-#pragma unroll
-    for (int v = 0; v < D / 8; ++v) {
-      float x[8];
-      unpack8<T>(__ldg(g + v), x);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) kr[v * 8 + i] = x[i];
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < D; ++c) kr[c] = 0.f;
-  }
-  const int b_first = skip_masked ? kt : 0;
-  for (int b0 = b_first; b0 < NB; b0 += 16) {
-    const int nb = min(16, NB - b0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < nb * D; i += 128)
-      (&qm[0][0])[i] = q_mean[((size_t)bh * NB + b0) * D + i];
-    __syncthreads();
-    for (int bb = 0; bb < nb; ++bb) {
-      float acc = 0.f;
-#pragma unroll
-      for (int c = 0; c < D; c += 4) {
-        const float4 m4 = *reinterpret_cast<const float4*>(&qm[bb][c]);
-        acc = __fmaf_rn(m4.x, kr[c], acc);
-        acc = __fmaf_rn(m4.y, kr[c + 1], acc);
-        acc = __fmaf_rn(m4.z, kr[c + 2], acc);
-        acc = __fmaf_rn(m4.w, kr[c + 3], acc);
-      }
-      corr[((size_t)bh * NB + b0 + bb) * Np + j] = acc;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
 // V, pass 1: per-channel amax over all tokens.  grid (nchunks, B*H), 256
 // threads; one 128-token chunk per block; float bits of |x| >= 0 are ordered
 // like unsigned integers, so atomicMax on the bits is exact.
@@ -315,6 +265,9 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
 // ---------------------------------------------------------------------------
 // Host-side launchers (called by the C ABI after validation).
 template <typename T, int D>
+cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st);  // corr.cu
+
+template <typename T, int D>
 static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
   const int BH = a.B * a.H;
   const int nchunks = a.NB;
@@ -325,9 +278,9 @@ static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
   k_smooth_quant<T, D><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
       static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
       a.q_scale, a.q_mean, a.k_i4, a.k_scale);
-  k_qk_corr<T, D><<<dim3(a.NB, BH), 128, 0, st>>>(static_cast<const T*>(a.k), a.q_mean, a.N,
-                                                  a.Np, a.NB, a.skip_masked_corr, a.qk_corr);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_qk_corr_t<T, D>(a, st);
 }
 
 cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st) {

@@ -21,6 +21,7 @@ struct QKArgs {
   float* k_mean;
   float* qk_corr;
   float* mean_part;        // scratch [B*H, NB, d]
+  void* qbar_split;        // scratch [3][B*H][NBc*128][d] in the input dtype (NBc = ceil(NB/128))
   int skip_masked_corr;    // 1: skip correction blocks a causal mask hides
 };
 
@@ -53,6 +54,13 @@ cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_debug_qk(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int Np, int d,
                             int32_t* s_out, cudaStream_t st);
+
+// General tiled tensor map: `rank` dims (innermost first, in elements), the
+// byte strides of dims 1..rank-1, the box (elements), element size 1/2/4 B and
+// a swizzle of 0, 64 or 128 bytes.  Out-of-range box elements read as zero.
+cudaError_t make_tmap(void* tmap_out, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, int elem_bytes,
+                      int swizzle_bytes);
 
 // Tensor-map creation through the driver entry point (no link-time libcuda).
 // Encodes a 2-D row-major uint8 tensor [rows, cols] with a box of
