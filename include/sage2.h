@@ -24,12 +24,17 @@
  *
  * Payload layouts (the quantized intermediates, all on the device)
  * ----------------------------------------------------------------
- *  q_i4   int8  [B,H,Np,d]   INT4 values in [-7,7] of Q - qbar_block, rows >= N are 0
+ *  q_i4   u8    [B,H,Np,d]   INT4 values in [-7,7] of Q - qbar_block, each stored as its
+ *                            e4m3 code (every integer in [-7,7] is exact in e4m3; zero is
+ *                            +0, code 0x00), rows >= N are 0.  The FP8 tensor path then
+ *                            multiplies the INT4 values exactly, at the 8-bit integer
+ *                            path's rate, and gives S as an fp32 integer.
  *  q_scale f32  [B,H,Np]     per-token scale amax/7 (0 for an all-zero row / pad)
  *  q_mean f32   [B,H,NB,d]   mean of each 128-row block of Q (valid rows only)
- *  k_i4   int8  [B,H,Np,d]   INT4 values of K - kbar, rows >= N are 0.  Rows are stored
- *                            KEY-INTERLEAVED inside each 128-row block: stored row n of a
- *                            block holds token 64*(n%2) + n/2 of that block.
+ *  k_i4   u8    [B,H,Np,d]   INT4 values of K - kbar as e4m3 codes (as q_i4), rows >= N
+ *                            are 0.  Rows are stored
+ *                            PERMUTED inside each 128-row block: stored row n of a block
+ *                            holds token 32*((n/2)%4) + 2*(n/8) + n%2 of that block.
  *  k_scale f32  [B,H,Np]     per-token scale
  *  k_mean f32   [B,H,d]      token mean of K
  *  qk_corr f32  [B,H,NB,Np]  q_mean[blk] . K[j] (raw K), 0 for j >= N
@@ -76,8 +81,8 @@ typedef enum { SAGE2_F16 = 0, SAGE2_BF16 = 1, SAGE2_F32 = 2 } sage2_dtype;
  * qk_corr[blk][j] = sum_c q_mean[blk][c] * K[j][c], fp32.
  */
 sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int B, int H, int N,
-                                   int d, int8_t* q_i4, float* q_scale, float* q_mean,
-                                   int8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
+                                   int d, uint8_t* q_i4, float* q_scale, float* q_mean,
+                                   uint8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
                                    sage2_stream_t stream);
 
 /*
@@ -96,13 +101,13 @@ sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d,
  *   o       : [B,H,N,d] written in `o_dtype` (SAGE2_F16, SAGE2_BF16 or SAGE2_F32).
  *   causal  : 0 or 1.   sm_scale : softmax scale (> 0, finite).
  * Per 128-key tile, in ascending order, with L = sm_scale*log2(e):
- *   x = (q_scale_i*k_scale_j*S_ij + qk_corr[blk(i)][j]) * L,  S = q_i4 . k_i4 (s32)
+ *   x = (q_scale_i*k_scale_j*S_ij + qk_corr[blk(i)][j]) * L,  S = q_i4 . k_i4 (exact)
  *   running max m, p = exp2(x - m), l += p, P~ = e4m3(448 p),
  *   inner = P~ . V~ over the tile (fresh fp32 accumulator),
  *   acc = alpha*acc + inner (alpha = exp2(m_old - m_new));  O = acc*v_scale/(448 l).
  */
-sage2_status sage2_attn_fwd_quantized(const int8_t* q_i4, const float* q_scale,
-                                      const int8_t* k_i4, const float* k_scale,
+sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
+                                      const uint8_t* k_i4, const float* k_scale,
                                       const float* qk_corr, const uint8_t* v_fp8_t,
                                       const float* v_scale, void* o, int o_dtype, int B, int H,
                                       int N, int d, int causal, float sm_scale,
@@ -144,12 +149,14 @@ size_t sage2_workspace_bytes(int B, int H, int N, int d);
 
 /*
  * Test entry: the raw integer products S = q_i4 . k_i4^T of every 128x128
- * tile, through the same TMA + tcgen05 kind::i8 path as the attention kernel.
+ * tile, through the same TMA + tcgen05 FP8 (kind::f8f6f4, fp32 accumulator)
+ * path as the attention kernel, converted to int32 (the fp32 sums are exact
+ * integers for INT4 operands).
  *   s_out : int32 [B,H,Np,Np] (caller-allocated).  Column j holds the product with
- *           stored k_i4 row j (so, with the key-interleaved k_i4 layout, key
- *           64*(j%2) + (j%128)/2 of block j/128).
+ *           stored k_i4 row j (so, with the permuted k_i4 layout, key
+ *           32*((j%128/2)%4) + 2*((j%128)/8) + j%2 of block j/128).
  */
-sage2_status sage2_debug_qk_s32(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int N,
+sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
                                 int d, int32_t* s_out, sage2_stream_t stream);
 
 /*

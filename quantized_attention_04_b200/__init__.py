@@ -118,9 +118,10 @@ def sage2_check_device_error(device=None) -> int:
     return int(lib().sage2_check_device_error(st))
 
 
-def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor) -> dict:
+def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = None) -> dict:
     """Smoothing + INT4 of Q and K and the Q-smoothing correction.
-    Returns the payload dict (q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr)."""
+    Returns the payload dict (q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
+    `out`, if given, is such a dict (from an earlier call) and is overwritten."""
     B, H, N, d = _dims(q)
     if k.shape != q.shape or k.dtype != q.dtype:
         raise ValueError("q and k must have the same shape and dtype")
@@ -128,15 +129,8 @@ def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor) -> dict:
     Np = n_pad(N)
     NB = Np // 128
     dev = q.device
-    out = dict(
-        q_i4=torch.empty(B, H, Np, d, dtype=torch.int8, device=dev),
-        q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
-        q_mean=torch.empty(B, H, NB, d, dtype=torch.float32, device=dev),
-        k_i4=torch.empty(B, H, Np, d, dtype=torch.int8, device=dev),
-        k_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
-        k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev),
-        qk_corr=torch.empty(B, H, NB, Np, dtype=torch.float32, device=dev),
-    )
+    if out is None:
+        out = _qk_payloads(B, H, Np, NB, d, dev)
     st = lib().sage2_smooth_quant_qk(
         _ptr(q), _ptr(k), _DT[q.dtype], B, H, N, d, _ptr(out["q_i4"]), _ptr(out["q_scale"]),
         _ptr(out["q_mean"]), _ptr(out["k_i4"]), _ptr(out["k_scale"]), _ptr(out["k_mean"]),
@@ -145,12 +139,28 @@ def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor) -> dict:
     return out
 
 
-def sage2_quant_v(v: torch.Tensor):
-    """FP8 e4m3 V per channel. Returns (v_fp8_t uint8 [B,H,d,Np], v_scale f32 [B,H,d])."""
+def _qk_payloads(B, H, Np, NB, d, dev) -> dict:
+    return dict(
+        q_i4=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),   # e4m3 codes of INT4 values
+        q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
+        q_mean=torch.empty(B, H, NB, d, dtype=torch.float32, device=dev),
+        k_i4=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),   # e4m3 codes, rows permuted per block
+        k_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
+        k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev),
+        qk_corr=torch.empty(B, H, NB, Np, dtype=torch.float32, device=dev),
+    )
+
+
+def sage2_quant_v(v: torch.Tensor, out: tuple | None = None):
+    """FP8 e4m3 V per channel. Returns (v_fp8_t uint8 [B,H,d,Np], v_scale f32 [B,H,d]);
+    `out`, if given, is such a pair (from an earlier call) and is overwritten."""
     B, H, N, d = _dims(v)
     Np = n_pad(N)
-    vt = torch.empty(B, H, d, Np, dtype=torch.uint8, device=v.device)
-    vs = torch.empty(B, H, d, dtype=torch.float32, device=v.device)
+    if out is None:
+        vt = torch.empty(B, H, d, Np, dtype=torch.uint8, device=v.device)
+        vs = torch.empty(B, H, d, dtype=torch.float32, device=v.device)
+    else:
+        vt, vs = out
     st = lib().sage2_quant_v(_ptr(v), _DT[v.dtype], B, H, N, d, _ptr(vt), _ptr(vs), _stream(v))
     _check("sage2_quant_v", st)
     return vt, vs
@@ -216,7 +226,8 @@ def sage2_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ca
 
 
 def sage2_debug_qk_s32(q_i4: torch.Tensor, k_i4: torch.Tensor, N: int) -> torch.Tensor:
-    """Raw int32 tiles of q_i4 . k_i4^T through the tcgen05 kind::i8 path."""
+    """Raw int32 tiles of q_i4 . k_i4^T (e4m3 codes of INT4 values) through the
+    tcgen05 FP8 path of the attention kernel."""
     B, H, Np, d = q_i4.shape
     s = torch.empty(B, H, Np, Np, dtype=torch.int32, device=q_i4.device)
     st = lib().sage2_debug_qk_s32(_ptr(q_i4), _ptr(k_i4), B, H, N, d, _ptr(s), _stream(q_i4))

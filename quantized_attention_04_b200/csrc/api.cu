@@ -173,8 +173,8 @@ using namespace sage2;
 extern "C" {
 
 sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int B, int H, int N,
-                                   int d, int8_t* q_i4, float* q_scale, float* q_mean,
-                                   int8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
+                                   int d, uint8_t* q_i4, float* q_scale, float* q_mean,
+                                   uint8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
                                    sage2_stream_t stream) {
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
@@ -220,8 +220,8 @@ sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d,
   return from_cuda(e != cudaSuccess ? e : e2);
 }
 
-sage2_status sage2_attn_fwd_quantized(const int8_t* q_i4, const float* q_scale,
-                                      const int8_t* k_i4, const float* k_scale,
+sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
+                                      const uint8_t* k_i4, const float* k_scale,
                                       const float* qk_corr, const uint8_t* v_fp8_t,
                                       const float* v_scale, void* o, int o_dtype, int B, int H,
                                       int N, int d, int causal, float sm_scale,
@@ -268,8 +268,8 @@ sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o
   e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), w.total, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
 
-  int8_t* q_i4 = reinterpret_cast<int8_t*>(ws + w.off_q_i4);
-  int8_t* k_i4 = reinterpret_cast<int8_t*>(ws + w.off_k_i4);
+  uint8_t* q_i4 = reinterpret_cast<uint8_t*>(ws + w.off_q_i4);
+  uint8_t* k_i4 = reinterpret_cast<uint8_t*>(ws + w.off_k_i4);
   uint8_t* vt = ws + w.off_vt;
   float* qs = reinterpret_cast<float*>(ws + w.off_qs);
   float* ks = reinterpret_cast<float*>(ws + w.off_ks);
@@ -292,7 +292,7 @@ sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o
   return from_cuda(e != cudaSuccess ? e : e2);
 }
 
-sage2_status sage2_debug_qk_s32(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int N,
+sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
                                 int d, int32_t* s_out, sage2_stream_t stream) {
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);

@@ -7,20 +7,21 @@
 // One CTA = one 128-row query block of one head; 384 threads, warp-specialised:
 //   warp 0        TMA producer: the Q^ tile once, then per key tile K^, V^T,
 //                 the key scales and the correction chunk (kStages-deep ring).
-//   warp 1        MMA issuer (one thread): S = Q^ K^T with tcgen05 kind::i8
-//                 into TMEM (s32, two buffers, issued two key tiles ahead), and
+//   warp 1        MMA issuer (one thread): S = Q^ K^T with tcgen05 kind::f8f6f4
+//                 (the INT4 values carried as e4m3 codes; exact fp32 integer
+//                 sums) into TMEM (two buffers, issued two key tiles ahead), and
 //                 inner = P~ V~ with kind::f8f6f4 (e4m3 -> f32) into a fresh
 //                 TMEM accumulator per key tile (two buffers).
 //   warp 2        TMEM allocator.
-//   warps 4-7,    two softmax warpgroups.  Thread (h, i) owns query row i (TMEM
-//   warps 8-11    lane i) and half h of every key tile: score columns
-//                 64h..64h+63 and output channels (d/2)h..(d/2)h+d/2-1.  Per
-//                 tile: dequantise + correct its 64 scores, publish the partial
-//                 row max, fold the previous tile's inner product into the
-//                 register accumulator (acc = alpha*acc + inner: the outer level
-//                 of the two-level accumulation) while the other half publishes,
-//                 then exp2, l, and P~ = e4m3(448 p) into shared memory (the
-//                 MMA's swizzled layout).
+//   warps 4-7,    two softmax warpgroups.  Warpgroup h owns lanes 16h..16h+15 of
+//   warps 8-11    every 32-lane TMEM quadrant; with .16x256b loads a thread owns
+//                 two query rows and 32 consecutive keys of each tile (four
+//                 threads of a warp share a row).  Per tile: fold the inner
+//                 product of tile t-2 into the register accumulator (acc =
+//                 alpha*acc + inner: the outer level of the two-level
+//                 accumulation), dequantise + correct its 64 scores, row max
+//                 across the four threads, exp2, l, and P~ = e4m3(448 p) into
+//                 shared memory (the MMA's swizzled layout).
 // TMEM columns: S[b] at 128*b (b = 0, 1), inner[b] at 256 + d*b.
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout the kernel
 // records it in the device error word and every role leaves its loop.
@@ -36,9 +37,8 @@ namespace sage2 {
 
 constexpr int kStages = 4;
 constexpr int kThreads = 384;
+constexpr int kSegStride = 36;                   // floats between the 32-key groups in shared memory
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
-constexpr uint32_t kMagicBits = 0x4B400000u;     // 1.5 * 2^23
-constexpr float kMagic = 12582912.0f;
 
 template <int D>
 struct __align__(1024) AttnSmem {
@@ -46,11 +46,11 @@ struct __align__(1024) AttnSmem {
   uint8_t k[kStages][128 * D];     // K^ tiles
   uint8_t v[kStages][D * 128];     // V^T tiles: D rows (channels) x 128 tokens
   uint8_t p[2][128 * 128];         // P~ tiles: 128 rows x 128 tokens (e4m3)
-  // qk_corr and k_scale of the key tile: keys 0-63 at [0, 64), keys 64-127 at
-  // [68, 132).  The 16-byte gap puts the two halves (read by the two column
-  // parities of a warp in the same instruction) in different banks.
-  float corr[kStages][136];
-  float ksc[kStages][136];
+  // qk_corr and k_scale of the key tile: keys 32g..32g+31 at [36g, 36g+32).
+  // The 16-byte gaps put the four groups (read by the four threads g of a
+  // row in the same instruction) in different banks.
+  float corr[kStages][4 * kSegStride];
+  float ksc[kStages][4 * kSegStride];
   float qsc[128];                  // q_scale of the block's rows
   float vsc[2][D];                 // v_scale (one copy per softmax warpgroup)
   uint64_t q_full;
@@ -89,40 +89,109 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Dequantise + correct 32 scores: x' = sq_i * (sk_j * S_ij) + C_j.  The s32
-// value plus 0x4B400000, read as a float, is exactly 1.5*2^23 + S
-// (|S| <= 49*128 < 2^22); subtracting 1.5*2^23 is exact.
-__device__ __forceinline__ void dequant32(const uint32_t (&sr)[32], const float* ck,
-                                          const float* kk, float2 a2, float* x) {
-  const float2 nm2 = make_float2(-kMagic, -kMagic);
+// Dequantise + correct the 16 keys 4m..4m+3 (m = 0..3) of both rows held in
+// one .16x256b.x8 load: x' = sq_i * (sk_j * S_ij) + C_j.  S comes out of the
+// FP8 tensor path as an fp32 integer: the INT4 values are exact in e4m3, every
+// product (|.| <= 49) and partial sum (|.| <= 49*128 < 2^13) is an integer the
+// fp32 accumulator holds exactly.
+__device__ __forceinline__ void dequant16(const uint32_t (&sr)[32], const float* ck,
+                                          const float* kk, float2 a0, float2 a1, float* x0,
+                                          float* x1) {
 #pragma unroll
-  for (int j = 0; j < 32; j += 4) {
-    const float4 c4 = *reinterpret_cast<const float4*>(ck + j);
-    const float4 k4 = *reinterpret_cast<const float4*>(kk + j);
-    float2 f0 = make_float2(__uint_as_float(sr[j] + kMagicBits), __uint_as_float(sr[j + 1] + kMagicBits));
-    float2 f1 = make_float2(__uint_as_float(sr[j + 2] + kMagicBits), __uint_as_float(sr[j + 3] + kMagicBits));
-    f0 = __fadd2_rn(f0, nm2);
-    f1 = __fadd2_rn(f1, nm2);
-    f0 = __fmul2_rn(make_float2(k4.x, k4.y), f0);
-    f1 = __fmul2_rn(make_float2(k4.z, k4.w), f1);
-    f0 = __ffma2_rn(a2, f0, make_float2(c4.x, c4.y));
-    f1 = __ffma2_rn(a2, f1, make_float2(c4.z, c4.w));
-    x[j] = f0.x;
-    x[j + 1] = f0.y;
-    x[j + 2] = f1.x;
-    x[j + 3] = f1.y;
+  for (int m = 0; m < 4; ++m) {
+    const float4 c4 = *reinterpret_cast<const float4*>(ck + 4 * m);
+    const float4 k4 = *reinterpret_cast<const float4*>(kk + 4 * m);
+    const float2 kxy = make_float2(k4.x, k4.y), kzw = make_float2(k4.z, k4.w);
+    const float2 cxy = make_float2(c4.x, c4.y), czw = make_float2(c4.z, c4.w);
+    const uint32_t* q = sr + 8 * m;
+    const float2 r00 = __ffma2_rn(a0, __fmul2_rn(kxy, make_float2(__uint_as_float(q[0]), __uint_as_float(q[1]))), cxy);
+    const float2 r01 = __ffma2_rn(a0, __fmul2_rn(kzw, make_float2(__uint_as_float(q[4]), __uint_as_float(q[5]))), czw);
+    const float2 r10 = __ffma2_rn(a1, __fmul2_rn(kxy, make_float2(__uint_as_float(q[2]), __uint_as_float(q[3]))), cxy);
+    const float2 r11 = __ffma2_rn(a1, __fmul2_rn(kzw, make_float2(__uint_as_float(q[6]), __uint_as_float(q[7]))), czw);
+    x0[4 * m] = r00.x;
+    x0[4 * m + 1] = r00.y;
+    x0[4 * m + 2] = r01.x;
+    x0[4 * m + 3] = r01.y;
+    x1[4 * m] = r10.x;
+    x1[4 * m + 1] = r10.y;
+    x1[4 * m + 2] = r11.x;
+    x1[4 * m + 3] = r11.y;
   }
 }
 
-// acc[32 channels] = alpha * acc + inner (the outer level of the accumulation).
-__device__ __forceinline__ void fold32(float* acc, const uint32_t (&in)[32], float al) {
-  const float2 al2 = make_float2(al, al);
+__device__ __forceinline__ float rowmax32(const float (&x)[32]) {
+  float m4[4];
 #pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    const float2 r = __ffma2_rn(al2, make_float2(acc[c], acc[c + 1]),
-                                make_float2(__uint_as_float(in[c]), __uint_as_float(in[c + 1])));
-    acc[c] = r.x;
-    acc[c + 1] = r.y;
+  for (int g = 0; g < 4; ++g)
+    m4[g] = max3f(max3f(x[8 * g], x[8 * g + 1], x[8 * g + 2]),
+                  max3f(x[8 * g + 3], x[8 * g + 4], x[8 * g + 5]), fmaxf(x[8 * g + 6], x[8 * g + 7]));
+  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+}
+
+// p448 = exp2(x' L + nb) for the 32 keys of one row, e4m3-rounded (RN,
+// saturating) and stored as two 16-byte chunks (keys 0-15, 16-31) of the
+// row's 128-byte line of P~: chunks 2g, 2g+1 of the line, XOR-swizzled by
+// `sw` (the row mod 8: the MMA's 128-byte swizzle).  Returns the row's sum
+// of the unrounded p448.
+__device__ __forceinline__ float exp_pack_store(const float (&x)[32], float2 L2, float2 nb,
+                                                uint8_t* prow, int g, int sw) {
+  float2 sumA = make_float2(0.f, 0.f), sumB = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = c * 16 + u * 4;
+      float2 e0 = __ffma2_rn(make_float2(x[j], x[j + 1]), L2, nb);
+      float2 e1 = __ffma2_rn(make_float2(x[j + 2], x[j + 3]), L2, nb);
+      e0.x = ex2(e0.x);
+      e0.y = ex2(e0.y);
+      e1.x = ex2(e1.x);
+      e1.y = ex2(e1.y);
+      sumA = __fadd2_rn(sumA, e0);
+      sumB = __fadd2_rn(sumB, e1);
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(e0, __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(e1, __NV_SATFINITE, __NV_E4M3);
+      w[u] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>(prow + (((2 * g + c) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  const float2 s2 = __fadd2_rn(sumA, sumB);
+  return s2.x + s2.y;
+}
+
+// acc = alpha * acc + inner (the outer level of the accumulation) for the
+// thread's two rows (alpha.x row r0, alpha.y row r0+8), reading inner from
+// TMEM at taddr with .16x256b loads (layout of acc: see the softmax role).
+template <int D>
+__device__ __forceinline__ void fold_inner(float (&acc)[D / 2], uint32_t taddr, float2 alpha) {
+  const float2 a0 = make_float2(alpha.x, alpha.x), a1 = make_float2(alpha.y, alpha.y);
+  uint32_t in[D / 2];
+  tmem_ld16x256_32(taddr, *reinterpret_cast<uint32_t(*)[32]>(in));
+  if (D == 128) tmem_ld16x256_32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(in + (D == 128 ? 32 : 0)));
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < D / 2; i += 4) {
+    const float2 r0 = __ffma2_rn(a0, make_float2(acc[i], acc[i + 1]),
+                                 make_float2(__uint_as_float(in[i]), __uint_as_float(in[i + 1])));
+    const float2 r1 = __ffma2_rn(a1, make_float2(acc[i + 2], acc[i + 3]),
+                                 make_float2(__uint_as_float(in[i + 2]), __uint_as_float(in[i + 3])));
+    acc[i] = r0.x;
+    acc[i + 1] = r0.y;
+    acc[i + 2] = r1.x;
+    acc[i + 3] = r1.y;
+  }
+}
+
+// Two adjacent output channels (index of the first, even) in the output type.
+template <int OT>
+__device__ __forceinline__ void store_pair(void* out, size_t idx, float f0, float f1) {
+  if (OT == 2) {
+    *reinterpret_cast<float2*>(static_cast<float*>(out) + idx) = make_float2(f0, f1);
+  } else if (OT == 0) {
+    *reinterpret_cast<__half2*>(static_cast<uint16_t*>(out) + idx) = __floats2half2_rn(f0, f1);
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(out) + idx) = __floats2bfloat162_rn(f0, f1);
   }
 }
 
@@ -136,7 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  constexpr int DH = D / 2;                       // output channels per softmax half
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = causal ? (NB - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
@@ -193,10 +261,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&sm.kv_full[s], 128 * D + D * 128 + 512 + 512);
         tma_load_2d(sm.k[s], &tm_k, &sm.kv_full[s], 0, bh * Np + t * 128);
         tma_load_2d(sm.v[s], &tm_v, &sm.kv_full[s], t * 128, bh * D);
-        bulk_load(sm.corr[s], corr_row + t * 128, 256, &sm.kv_full[s]);
-        bulk_load(sm.corr[s] + 68, corr_row + t * 128 + 64, 256, &sm.kv_full[s]);
-        bulk_load(sm.ksc[s], ks_row + t * 128, 256, &sm.kv_full[s]);
-        bulk_load(sm.ksc[s] + 68, ks_row + t * 128 + 64, 256, &sm.kv_full[s]);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          bulk_load(sm.corr[s] + kSegStride * g, corr_row + t * 128 + 32 * g, 128, &sm.kv_full[s]);
+          bulk_load(sm.ksc[s] + kSegStride * g, ks_row + t * 128 + 32 * g, 128, &sm.kv_full[s]);
+        }
       }
       if (*abort_flag) {
         // let the copies already issued land before the block exits
@@ -208,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_i8_s32(128, 128);
+      constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128);   // INT4 values in e4m3
       constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, D);
       // descriptors are built once; a k-step or a stage only moves the start
       // address field (16-byte units; shared memory is < 256 KB, no carry)
@@ -227,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t kb = dk + s * kStageK;
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk) mma_i8_ss(tmem + b * 128, dq + 2 * kk, kb + 2 * kk, idesc_qk, kk > 0);
+        for (int kk = 0; kk < D / 32; ++kk) mma_f8_ss(tmem + b * 128, dq + 2 * kk, kb + 2 * kk, idesc_qk, kk > 0);
         tc_commit(&sm.s_full[b]);
         return true;
       };
@@ -262,31 +331,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Raised inside the branch it governs, so that the compiler allocates this
     // role's code against the larger budget (40*128 + 232*256 <= 168*384).
     setmaxnreg_inc<232>();
-    // The .16x64b TMEM loads give thread t of a warp lane (t>>2) + 8*(t&1) of
-    // a 16-lane group and every other column, parity (t>>1)&1.  Warpgroup h
-    // takes lanes 16h..16h+15 of each 32-lane quadrant, so every query row is
-    // owned by the two threads t and t^2 of one warp.  With the key-interleaved
-    // K^ layout, the score columns of parity `par` are the 64 consecutive keys
-    // 64*par .. 64*par+63 of the tile, and the inner-product columns of parity
-    // `par` are the output channels 2k + par.
+    // The .16x256b TMEM loads give thread t of a warp, in a 16-lane group, the
+    // two lanes t/4 and t/4 + 8 and the columns 8k + 2g + {0,1} (g = t%4,
+    // k = 0..15).  Warpgroup h takes lanes 16h..16h+15 of each 32-lane
+    // quadrant, so every query row is shared by the four threads g = 0..3 of
+    // one warp and each thread owns two rows.  With the K^ rows of each block
+    // stored so that column 8k + 2g + e holds token 32g + 2k + e, thread g sees
+    // the 32 consecutive keys 32g..32g+31 of the tile (both rows), and the
+    // inner-product columns it loads are output channels 8k + 2g + {0,1}.
     const int h = wg - 1;
     const int quad = warp & 3;
-    const int par = (lane >> 1) & 1;
-    const int r = 32 * quad + 16 * h + (lane >> 2) + 8 * (lane & 1);   // row in the block
-    const int row = qt * 128 + r;                                       // row in the head
+    const int g = lane & 3;
+    const int r0 = 32 * quad + 16 * h + (lane >> 2);      // rows in the block: r0, r0 + 8
+    const int row0 = qt * 128 + r0, row1 = row0 + 8;      // rows in the head
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quad + 16 * h) << 16;
     const uint32_t tS = tmem + lane_addr;                 // + 128*b: S buffer b
     const uint32_t tI = tmem + lane_addr + 256;           // + D*b: inner buffer b
     for (int i = threadIdx.x - 128 * wg; i < D; i += 128)
       sm.vsc[h][i] = v_scale[static_cast<size_t>(bh) * D + i];
     named_bar_sync(1 + h, 128);
-    float acc[DH];                                        // channels 2k + par
+    // acc[4k + e] / acc[4k + 2 + e]: rows r0 / r0+8, channel 8k + 2g + e
+    // (k < 8; channels 64 + ... in the second half when D = 128)
+    float acc[D / 2];
 #pragma unroll
-    for (int c = 0; c < DH; ++c) acc[c] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    for (int c = 0; c < D / 2; ++c) acc[c] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float2 al_1 = make_float2(0.f, 0.f), al_2 = make_float2(0.f, 0.f);  // (row0, row1) alpha of tiles t-1, t-2
     bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag);
-    const float a = ok ? sm.qsc[r] : 0.f;
-    const float2 a2 = make_float2(a, a);
+    const float a0 = ok ? sm.qsc[r0] : 0.f, a1 = ok ? sm.qsc[r0 + 8] : 0.f;
+    const float2 a02 = make_float2(a0, a0), a12 = make_float2(a1, a1);
     const float2 L2 = make_float2(L, L);
     // the second warpgroup starts half a tile late, so that one group's exp2
     // phase overlaps the other group's dequantisation
@@ -294,145 +367,86 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int t = 0; ok && t < nt; ++t) {
       const int s = t % kStages, b = t & 1;
+      // s_full(t) also says PV(t-2) is complete: the MMA thread issued QK(t)
+      // after PV(t-2), and the commit tracks every earlier MMA.  So inner(t-2)
+      // can be folded now and P~[b] is free, with no wait of their own.
       if (!mbar_wait_warp(&sm.s_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float x[64];                                        // keys 64*par + k
+      if (t >= 2) fold_inner<D>(acc, tI + b * D, al_2);   // outer level for tile t-2
+      float x0[32], x1[32];                               // rows r0, r0+8; keys 32g + j
       {
-        uint32_t s0[32], s1[32];
-        tmem_ld16x64_32(tS + b * 128, s0);
-        tmem_ld16x64_32(tS + b * 128 + 64, s1);
+        uint32_t sA[32], sB[32];
+        tmem_ld16x256_32(tS + b * 128, sA);
+        tmem_ld16x256_32(tS + b * 128 + 64, sB);
         tmem_ld_wait();
         // the key scales and correction chunk of stage s are visible: s_full
         // also carries the MMA thread's release after it acquired kv_full
-        dequant32(s0, sm.corr[s] + 68 * par, sm.ksc[s] + 68 * par, a2, x);
-        dequant32(s1, sm.corr[s] + 68 * par + 32, sm.ksc[s] + 68 * par + 32, a2, x + 32);
+        const float* ck = sm.corr[s] + kSegStride * g;
+        const float* kk = sm.ksc[s] + kSegStride * g;
+        dequant16(sA, ck, kk, a02, a12, x0, x1);
+        dequant16(sB, ck + 16, kk + 16, a02, a12, x0 + 16, x1 + 16);
       }
       if ((causal && t == qt) || (tail && t == NB - 1)) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const int key = t * 128 + 64 * par + k;
-          if (key >= N || (causal && key > row)) x[k] = -INFINITY;
+        for (int j = 0; j < 32; ++j) {
+          const int key = t * 128 + 32 * g + j;
+          if (key >= N || (causal && key > row0)) x0[j] = -INFINITY;
+          if (key >= N || (causal && key > row1)) x1[j] = -INFINITY;
         }
       }
-      float mx8[8];
-#pragma unroll
-      for (int g = 0; g < 8; ++g)
-        mx8[g] = max3f(max3f(x[8 * g], x[8 * g + 1], x[8 * g + 2]),
-                       max3f(x[8 * g + 3], x[8 * g + 4], x[8 * g + 5]),
-                       fmaxf(x[8 * g + 6], x[8 * g + 7]));
-      float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
-                       fmaxf(mx8[6], mx8[7]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));   // the row's other half
+      float mx0 = rowmax32(x0), mx1 = rowmax32(x1);
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));   // the rows' other threads
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
       if (h == 0 && t == 0) { __syncwarp(); if (lane == 0) mbar_arrive(&sm.offset_bar); }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = ex2((m - m_new) * L);           // 0 on the first tile
-      const float base = m_new * L - kLog2_448;           // p448 = 448 * exp2((x'-m)L)
-      const float2 nb2 = make_float2(-base, -base);
-      // the P~ buffer of this parity is free: PV(t-2) completed before i_full of
-      // tile t-2 fired, which this thread waited for in the previous tile
-      uint8_t* prow = sm.p[b] + r * 128;
-      float2 sumA = make_float2(0.f, 0.f), sumB = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = c * 16 + u * 4;
-          float2 e0 = __ffma2_rn(make_float2(x[j], x[j + 1]), L2, nb2);
-          float2 e1 = __ffma2_rn(make_float2(x[j + 2], x[j + 3]), L2, nb2);
-          e0.x = ex2(e0.x);
-          e0.y = ex2(e0.y);
-          e1.x = ex2(e1.x);
-          e1.y = ex2(e1.y);
-          sumA = __fadd2_rn(sumA, e0);
-          sumB = __fadd2_rn(sumB, e1);
-          const uint32_t lo = __nv_cvt_float2_to_fp8x2(e0, __NV_SATFINITE, __NV_E4M3);
-          const uint32_t hi = __nv_cvt_float2_to_fp8x2(e1, __NV_SATFINITE, __NV_E4M3);
-          w[u] = lo | (hi << 16);
-        }
-        const int chunk = 4 * par + c;                    // 16-byte chunk of the 128-byte row
-        *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float2 alpha = make_float2(ex2((m0 - mn0) * L), ex2((m1 - mn1) * L));  // 0 on the first tile
+      // p448 = 448 * exp2((x' - m) L) = exp2(x' L - (m L - log2 448))
+      const float2 nb0 = make_float2(kLog2_448 - mn0 * L, kLog2_448 - mn0 * L);
+      const float2 nb1 = make_float2(kLog2_448 - mn1 * L, kLog2_448 - mn1 * L);
+      // the P~ buffer of this parity is free: PV(t-2) completed (see s_full above)
+      uint8_t* p0 = sm.p[b] + r0 * 128;
+      uint8_t* p1 = p0 + 8 * 128;
+      const float s0 = exp_pack_store(x0, L2, nb0, p0, g, r0 & 7);
+      const float s1 = exp_pack_store(x1, L2, nb1, p1, g, r0 & 7);
       fence_proxy_async_smem();
       tc_fence_before();                                  // S(t) and inner(t-2) reads are done
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[b]);
-      const float2 sum2 = __fadd2_rn(sumA, sumB);
-      l = alpha * l + (sum2.x + sum2.y);
-      m = m_new;
-
-      // outer level for the previous tile, whose PV product ran meanwhile
-      if (t >= 1) {
-        const int u = t - 1, ub = u & 1;
-        if (!mbar_wait_warp(&sm.i_full[ub], (u >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t in0[32], in1[32];
-        tmem_ld16x64_32(tI + ub * D, in0);
-        if (DH == 64) tmem_ld16x64_32(tI + ub * D + 64, in1);
-        tmem_ld_wait();
-        fold32(acc, in0, alpha_prev);
-        if (DH == 64) fold32(acc + (DH == 64 ? 32 : 0), in1, alpha_prev);
-      }
-      alpha_prev = alpha;
+      l0 = alpha.x * l0 + s0;
+      l1 = alpha.y * l1 + s1;
+      m0 = mn0;
+      m1 = mn1;
+      al_2 = al_1;
+      al_1 = alpha;
     }
     if (ok) {
+      // the last one or two inner products: i_full of the last tile's PV covers
+      // every MMA issued before it
       const int u = nt - 1, ub = u & 1;
       ok = mbar_wait_warp(&sm.i_full[ub], (u >> 1) & 1, abort_flag);
       if (ok) {
         tc_fence_after();
-        uint32_t in0[32], in1[32];
-        tmem_ld16x64_32(tI + ub * D, in0);
-        if (DH == 64) tmem_ld16x64_32(tI + ub * D + 64, in1);
-        tmem_ld_wait();
-        fold32(acc, in0, alpha_prev);
-        if (DH == 64) fold32(acc + (DH == 64 ? 32 : 0), in1, alpha_prev);
+        if (nt >= 2) fold_inner<D>(acc, tI + (ub ^ 1) * D, al_2);
+        fold_inner<D>(acc, tI + ub * D, al_1);
       }
     }
     if (ok) {
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      const float inv_l = 1.0f / l;
-      // swap half of the channels with the row's other thread so that each
-      // thread holds D/2 consecutive output channels: (D/2)*par + i
-      float o[DH];
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      const float inv0 = 1.0f / l0, inv1 = 1.0f / l1;
+      const float* vs = sm.vsc[h];
 #pragma unroll
-      for (int i = 0; i < DH / 2; ++i) {
-        const float send = par ? acc[i] : acc[DH / 2 + i];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-        const float own = par ? acc[DH / 2 + i] : acc[i];
-        o[2 * i] = par ? recv : own;
-        o[2 * i + 1] = par ? own : recv;
-      }
-      if (row < N) {
-        const float* vs = sm.vsc[h] + DH * par;
-        const size_t obase = (static_cast<size_t>(bh) * N + row) * D + DH * par;
-        if (OT == 2) {
-          float* op = static_cast<float*>(out) + obase;
-#pragma unroll
-          for (int c = 0; c < DH; c += 4) {
-            *reinterpret_cast<float4*>(op + c) =
-                make_float4(o[c] * vs[c] * inv_l, o[c + 1] * vs[c + 1] * inv_l,
-                            o[c + 2] * vs[c + 2] * inv_l, o[c + 3] * vs[c + 3] * inv_l);
-          }
-        } else {
-          uint16_t* op = static_cast<uint16_t*>(out) + obase;
-#pragma unroll
-          for (int c = 0; c < DH; c += 8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float f0 = o[c + 2 * u] * vs[c + 2 * u] * inv_l;
-              const float f1 = o[c + 2 * u + 1] * vs[c + 2 * u + 1] * inv_l;
-              if (OT == 0) {
-                const __half2 hv = __floats2half2_rn(f0, f1);
-                w[u] = *reinterpret_cast<const uint32_t*>(&hv);
-              } else {
-                const __nv_bfloat162 hv = __floats2bfloat162_rn(f0, f1);
-                w[u] = *reinterpret_cast<const uint32_t*>(&hv);
-              }
-            }
-            *reinterpret_cast<uint4*>(op + c) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+      for (int i = 0; i < D / 2; i += 4) {
+        const int c = 8 * ((i >> 2) & 7) + 2 * g + 64 * (i >> 5);   // channel of acc[i], acc[i+1]
+        const float v0 = vs[c], v1 = vs[c + 1];
+        if (row0 < N) store_pair<OT>(out, (static_cast<size_t>(bh) * N + row0) * D + c,
+                                     acc[i] * v0 * inv0, acc[i + 1] * v1 * inv0);
+        if (row1 < N) store_pair<OT>(out, (static_cast<size_t>(bh) * N + row1) * D + c,
+                                     acc[i + 2] * v0 * inv1, acc[i + 3] * v1 * inv1);
       }
     }
   }

@@ -1,5 +1,6 @@
-// Test kernel: raw s32 tiles of the INT4 product Q^ K^T through the same TMA +
-// tcgen05 kind::i8 path as the attention kernel (one 128x128 tile per CTA).
+// Test kernel: raw tiles of the INT4 product Q^ K^T through the same TMA +
+// tcgen05 FP8 path as the attention kernel (INT4 values in e4m3 codes, fp32
+// accumulator; one 128x128 tile per CTA), written as int32.
 // Lets the integer matrix product ("4-bit matrix multiplication", SageAttention2
 // abstract page, Abstract) be checked bit for bit on its own.
 #include <cuda.h>
@@ -45,10 +46,10 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
     tma_load_2d(sk, &tm_k, &bar_load, 0, bh * Np + kt * 128);
     if (mbar_wait(&bar_load, 0, &abort_flag)) {
       tc_fence_after();
-      constexpr uint32_t idesc = idesc_i8_s32(128, 128);
+      constexpr uint32_t idesc = idesc_e4m3_f32(128, 128);
 #pragma unroll
       for (int kk = 0; kk < D / 32; ++kk)
-        mma_i8_ss(tmem, smem_desc_kmajor(sq + 32 * kk, D), smem_desc_kmajor(sk + 32 * kk, D),
+        mma_f8_ss(tmem, smem_desc_kmajor(sq + 32 * kk, D), smem_desc_kmajor(sk + 32 * kk, D),
                   idesc, kk > 0);
       tc_commit(&bar_mma);
     }
@@ -66,7 +67,9 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
       tmem_ld_wait();
 #pragma unroll
       for (int u = 0; u < 32; u += 4)
-        *reinterpret_cast<int4*>(dst + c0 + u) = make_int4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+        *reinterpret_cast<int4*>(dst + c0 + u) =
+            make_int4(__float2int_rn(__uint_as_float(v[u])), __float2int_rn(__uint_as_float(v[u + 1])),
+                      __float2int_rn(__uint_as_float(v[u + 2])), __float2int_rn(__uint_as_float(v[u + 3])));
     }
   }
   tc_fence_before();
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
 }
 
 template <int D>
-static cudaError_t launch_debug_t(const int8_t* q_i4, const int8_t* k_i4, int BH, int Np,
+static cudaError_t launch_debug_t(const uint8_t* q_i4, const uint8_t* k_i4, int BH, int Np,
                                   int32_t* s_out, cudaStream_t st) {
   alignas(64) CUtensorMap tq, tk;
   cudaError_t e = make_tmap_u8_2d(&tq, q_i4, static_cast<uint64_t>(BH) * Np, D, 128, D);
@@ -91,7 +94,7 @@ static cudaError_t launch_debug_t(const int8_t* q_i4, const int8_t* k_i4, int BH
   return cudaGetLastError();
 }
 
-cudaError_t launch_debug_qk(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int Np, int d,
+cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int Np, int d,
                             int32_t* s_out, cudaStream_t st) {
   return d == 64 ? launch_debug_t<64>(q_i4, k_i4, B * H, Np, s_out, st)
                  : launch_debug_t<128>(q_i4, k_i4, B * H, Np, s_out, st);

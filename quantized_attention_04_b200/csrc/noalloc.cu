@@ -86,8 +86,8 @@ extern "C" sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, con
   if (ws == nullptr) return SAGE2_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-  int8_t* q_i4 = reinterpret_cast<int8_t*>(ws + w.off_q_i4);
-  int8_t* k_i4 = reinterpret_cast<int8_t*>(ws + w.off_k_i4);
+  uint8_t* q_i4 = reinterpret_cast<uint8_t*>(ws + w.off_q_i4);
+  uint8_t* k_i4 = reinterpret_cast<uint8_t*>(ws + w.off_k_i4);
   uint8_t* vt = ws + w.off_vt;
   float* qs = reinterpret_cast<float*>(ws + w.off_qs);
   float* ks = reinterpret_cast<float*>(ws + w.off_ks);

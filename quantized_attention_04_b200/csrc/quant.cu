@@ -107,8 +107,8 @@ __global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_smooth_quant(
     const T* __restrict__ q, const T* __restrict__ k, int N, int Np, int NB,
-    const float* __restrict__ kmean, int8_t* __restrict__ q_i4, float* __restrict__ q_scale,
-    float* __restrict__ q_mean, int8_t* __restrict__ k_i4, float* __restrict__ k_scale) {
+    const float* __restrict__ kmean, uint8_t* __restrict__ q_i4, float* __restrict__ q_scale,
+    float* __restrict__ q_mean, uint8_t* __restrict__ k_i4, float* __restrict__ k_scale) {
   __shared__ __align__(16) T tile[128][D];
   __shared__ float mean[D];
   const int blk = blockIdx.x, bh = blockIdx.y;
@@ -138,12 +138,13 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   }
   __syncthreads();
 
-  int8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * D;
+  uint8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * D;
   float* scale = (is_q ? q_scale : k_scale) + (size_t)bh * Np + r0;
-  // K^ rows are stored key-interleaved inside each 128-row block: token j of
-  // the block goes to stored row 2*(j % 64) + j / 64, so that stored row n
-  // holds token 64*(n % 2) + n / 2 (the attention kernel's TMEM loads then give
-  // each thread 64 consecutive keys).  Q^ rows keep their natural order.
+  // K^ rows are stored permuted inside each 128-row block: token j of the block
+  // goes to stored row 8*((j/2) % 16) + 2*(j/32) + j % 2, so that stored row n
+  // holds token 32*((n/2) % 4) + 2*(n/8) + n % 2 (the attention kernel's
+  // .16x256b TMEM loads then give each thread 32 consecutive keys).  Q^ rows
+  // keep their natural order.
   constexpr int CPL = D / 32;  // channels per lane: 4 (D=128) or 2 (D=64)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int r = warp; r < 128; r += 8) {
@@ -157,6 +158,10 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // Each INT4 value is stored as its e4m3 code: every integer in [-7, 7] is
+    // exact in e4m3, so the FP8 tensor path multiplies the INT4 values exactly
+    // (at the same rate as the 8-bit integer path) and yields S as an fp32
+    // integer.  Zero is stored as +0 (code 0x00).
     uint32_t packed = 0;
     float sc = 0.f;
     if (amax > 0.f) {
@@ -166,10 +171,12 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
       for (int i = 0; i < CPL; ++i) {
         float v = rintf(__fmul_rn(x[i], inv));
         v = fminf(fmaxf(v, -7.f), 7.f);
-        packed |= (static_cast<uint32_t>(static_cast<int>(v)) & 0xFFu) << (8 * i);
+        const float vi = static_cast<float>(static_cast<int>(v));   // -0 -> +0
+        packed |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(vi, __NV_SATFINITE, __NV_E4M3))
+                  << (8 * i);
       }
     }
-    const int srow = is_q ? r : 2 * (r & 63) + (r >> 6);
+    const int srow = is_q ? r : 8 * ((r >> 1) & 15) + 2 * (r >> 5) + (r & 1);
     if (CPL == 4) {
       reinterpret_cast<uint32_t*>(out + (size_t)srow * D)[lane] = packed;
     } else {

@@ -13,10 +13,10 @@ struct QKArgs {
   const void* k;
   int dtype;  // 0 fp16, 1 bf16
   int B, H, N, d, Np, NB;
-  int8_t* q_i4;
+  uint8_t* q_i4;
   float* q_scale;
   float* q_mean;
-  int8_t* k_i4;
+  uint8_t* k_i4;
   float* k_scale;
   float* k_mean;
   float* qk_corr;
@@ -35,9 +35,9 @@ struct VArgs {
 };
 
 struct AttnArgs {
-  const int8_t* q_i4;
+  const uint8_t* q_i4;
   const float* q_scale;
-  const int8_t* k_i4;
+  const uint8_t* k_i4;
   const float* k_scale;
   const float* qk_corr;
   const uint8_t* v_fp8_t;
@@ -52,7 +52,7 @@ struct AttnArgs {
 cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
-cudaError_t launch_debug_qk(const int8_t* q_i4, const int8_t* k_i4, int B, int H, int Np, int d,
+cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int Np, int d,
                             int32_t* s_out, cudaStream_t st);
 
 // General tiled tensor map: `rank` dims (innermost first, in elements), the

@@ -78,13 +78,26 @@ def bits_equal(a: np.ndarray, b: np.ndarray) -> bool:
     return np.array_equal(a, b)
 
 
+def int4_codes(i) -> np.ndarray:
+    """The library stores each INT4 value as its e4m3 code: the oracle's
+    integers encoded with the oracle's own (pinned) e4m3 codec."""
+    return orc.e4m3_encode(np.asarray(i, np.float64))
+
+
+def int4_values(codes) -> np.ndarray:
+    """INT4 values back from the library's e4m3 codes (must be integers in [-7, 7])."""
+    v = orc.e4m3_decode(np.asarray(codes, np.uint8))
+    assert np.array_equal(v, np.rint(v)) and np.abs(v).max(initial=0) <= 7
+    return v.astype(np.int8)
+
+
 def key_interleave(Np: int) -> np.ndarray:
-    """Index map of the library's key-interleaved k_i4 row order: stored row n
-    of each 128-row block holds token 64*(n % 2) + n // 2 of that block, so
-    stored = natural[key_interleave(Np)]."""
+    """Index map of the library's permuted k_i4 row order: stored row n of each
+    128-row block holds token 32*((n//2) % 4) + 2*(n//8) + n % 2 of that block,
+    so stored = natural[key_interleave(Np)]."""
     n = np.arange(Np)
     blk, j = n // 128, n % 128
-    return blk * 128 + 64 * (j % 2) + j // 2
+    return blk * 128 + 32 * ((j // 2) % 4) + 2 * (j // 8) + j % 2
 
 
 def default_scale(d: int) -> float:

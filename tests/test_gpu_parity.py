@@ -57,6 +57,7 @@ def test_payloads_bit_exact(qa, cfg):
             K = P.np32(k[b, h])
             o = orc.smooth_quant_qk(P.np32(q[b, h]), K)
             o["k_i4"] = o["k_i4"][P.key_interleave(Np)]       # the library's row order
+            o["q_i4"], o["k_i4"] = P.int4_codes(o["q_i4"]), P.int4_codes(o["k_i4"])
             for name in ("q_i4", "q_scale", "q_mean", "k_i4", "k_scale", "k_mean"):
                 assert P.bits_equal(g[name][b, h], o[name]), (name, b, h)
             ovt, ovs = orc.quant_v(P.np32(v[b, h]))
@@ -74,7 +75,7 @@ def test_qk_s32_bit_exact(qa, cfg):
     q, k, v, qd, kd, vd = _cuda(cfg)
     pay = qa.sage2_smooth_quant_qk(qd, kd)
     s = qa.sage2_debug_qk_s32(pay["q_i4"], pay["k_i4"], cfg.N).cpu().numpy()
-    qi, ki = pay["q_i4"].cpu().numpy(), pay["k_i4"].cpu().numpy()
+    qi, ki = P.int4_values(pay["q_i4"].cpu().numpy()), P.int4_values(pay["k_i4"].cpu().numpy())
     for b in range(cfg.B):
         for h in range(cfg.H):
             ref = orc.qk_int(qi[b, h], ki[b, h])        # columns follow the stored k_i4 rows
@@ -87,13 +88,18 @@ def test_qk_s32_bit_exact(qa, cfg):
 
 
 def test_qk_s32_on_oracle_payloads(qa):
-    """Oracle-made INT4 values (not the GPU's) through the integer MMA path."""
+    """Oracle-made INT4 values (not the GPU's) through the MMA path, including
+    the extreme products: all +-7 rows give |S| = 49*d."""
     rng = np.random.default_rng(31)
     for d in (64, 128):
         Np = 384
         qi = rng.integers(-7, 8, (1, 2, Np, d)).astype(np.int8)
         ki = rng.integers(-7, 8, (1, 2, Np, d)).astype(np.int8)
-        s = qa.sage2_debug_qk_s32(torch.from_numpy(qi).cuda(), torch.from_numpy(ki).cuda(), Np)
+        qi[0, 0, :128] = 7
+        ki[0, 0, :64] = 7
+        ki[0, 0, 64:128] = -7
+        s = qa.sage2_debug_qk_s32(torch.from_numpy(P.int4_codes(qi)).cuda(),
+                                  torch.from_numpy(P.int4_codes(ki)).cuda(), Np)
         s = s.cpu().numpy()
         for h in range(2):
             assert np.array_equal(s[0, h].astype(np.int64), orc.qk_int(qi[0, h], ki[0, h]))
@@ -160,6 +166,7 @@ def test_attention_config_sampled(qa, name):
     for b, h in heads:
         opay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, q_blocks=blocks)
         opay["k_i4"] = opay["k_i4"][P.key_interleave(opay["k_i4"].shape[0])]
+        opay["q_i4"], opay["k_i4"] = P.int4_codes(opay["q_i4"]), P.int4_codes(opay["k_i4"])
         for n in ("q_i4", "q_scale", "k_i4", "k_scale", "k_mean"):
             assert P.bits_equal(pay[n][b, h].cpu().numpy(), opay[n]), (name, n)
         got = P.np32(o[b, h])[rows]
