@@ -62,7 +62,6 @@ struct __align__(1024) AttnSmem {
                                     // says S[b] was read and inner[b] of tile t-2 folded
   uint64_t i_full[2];               // inner[b] written (tcgen05.commit)
   uint64_t drain;
-  uint64_t offset_bar;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -88,6 +87,13 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barriers of the exp2 ping-pong between the two softmax warps of one
+// SM sub-partition (quadrant q): kBarExpA + q is released by the second
+// warpgroup for the first, kBarExpB + q the other way round.
+constexpr int kBarExpA = 3, kBarExpB = 7;
 
 // Dequantise + correct the 16 keys 4m..4m+3 (m = 0..3) of both rows held in
 // one .16x256b.x8 load: x' = sq_i * (sk_j * S_ij) + C_j.  S comes out of the
@@ -225,7 +231,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.i_full[b], 1);
     }
     mbar_init(&sm.drain, 1);
-    mbar_init(&sm.offset_bar, 4);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -361,16 +366,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float a0 = ok ? sm.qsc[r0] : 0.f, a1 = ok ? sm.qsc[r0 + 8] : 0.f;
     const float2 a02 = make_float2(a0, a0), a12 = make_float2(a1, a1);
     const float2 L2 = make_float2(L, L);
-    // the second warpgroup starts half a tile late, so that one group's exp2
-    // phase overlaps the other group's dequantisation
-    if (ok && h == 1) ok = mbar_wait_warp(&sm.offset_bar, 0, abort_flag);
+    // The exp2 phases of the two warps that share an SM sub-partition (warp q
+    // of each warpgroup) take turns: one warp's exp2 runs while the other
+    // dequantises, so the MUFU is not split between them.  Every tile runs
+    // the full barrier protocol, also after a failed wait (the work is then
+    // skipped), so that neither warp can be left waiting on the other.
+    const int bar_mine = (h == 0 ? kBarExpA : kBarExpB) + quad;
+    const int bar_other = (h == 0 ? kBarExpB : kBarExpA) + quad;
 
-    for (int t = 0; ok && t < nt; ++t) {
+    for (int t = 0; t < nt; ++t) {
       const int s = t % kStages, b = t & 1;
       // s_full(t) also says PV(t-2) is complete: the MMA thread issued QK(t)
       // after PV(t-2), and the commit tracks every earlier MMA.  So inner(t-2)
       // can be folded now and P~[b] is free, with no wait of their own.
-      if (!mbar_wait_warp(&sm.s_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (ok) ok = mbar_wait_warp(&sm.s_full[b], (t >> 1) & 1, abort_flag);
+      if (!ok) {
+        if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
+        named_bar_arrive(bar_other, 64);
+        continue;
+      }
       tc_fence_after();
       if (t >= 2) fold_inner<D>(acc, tI + b * D, al_2);   // outer level for tile t-2
       float x0[32], x1[32];                               // rows r0, r0+8; keys 32g + j
@@ -399,17 +413,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      if (h == 0 && t == 0) { __syncwarp(); if (lane == 0) mbar_arrive(&sm.offset_bar); }
       const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
       const float2 alpha = make_float2(ex2((m0 - mn0) * L), ex2((m1 - mn1) * L));  // 0 on the first tile
       // p448 = 448 * exp2((x' - m) L) = exp2(x' L - (m L - log2 448))
       const float2 nb0 = make_float2(kLog2_448 - mn0 * L, kLog2_448 - mn0 * L);
       const float2 nb1 = make_float2(kLog2_448 - mn1 * L, kLog2_448 - mn1 * L);
+      // exp2 turn: the first warpgroup waits for the second one's previous tile,
+      // the second one for the first one's current tile
+      if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
       // the P~ buffer of this parity is free: PV(t-2) completed (see s_full above)
       uint8_t* p0 = sm.p[b] + r0 * 128;
       uint8_t* p1 = p0 + 8 * 128;
       const float s0 = exp_pack_store(x0, L2, nb0, p0, g, r0 & 7);
       const float s1 = exp_pack_store(x1, L2, nb1, p1, g, r0 & 7);
+      named_bar_arrive(bar_other, 64);
       fence_proxy_async_smem();
       tc_fence_before();                                  // S(t) and inner(t-2) reads are done
       __syncwarp();
@@ -421,6 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       al_2 = al_1;
       al_1 = alpha;
     }
+    // the second warpgroup's last turn ended
+    if (h == 0 && nt > 0) named_bar_sync(bar_mine, 64);
     if (ok) {
       // the last one or two inner products: i_full of the last tile's PV covers
       // every MMA issued before it
