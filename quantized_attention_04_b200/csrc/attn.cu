@@ -36,7 +36,7 @@
 namespace sage2 {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kSegStride = 36;                   // floats between the 32-key groups in shared memory
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 
@@ -52,7 +52,9 @@ struct __align__(1024) AttnSmem {
   float corr[kStages][4 * kSegStride];
   float ksc[kStages][4 * kSegStride];
   float qsc[128];                  // q_scale of the block's rows
-  float vsc[2][D];                 // v_scale (one copy per softmax warpgroup)
+  float vsc[D];                     // v_scale (correction warpgroup)
+  float alpha[4][128];              // per-row rescale factor of tile t in slot t%4 (softmax -> correction)
+  float lsum[128];                  // final row sums (448-scaled), softmax -> correction
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2];               // two arrivals: the MMA thread once it saw the key
@@ -60,7 +62,10 @@ struct __align__(1024) AttnSmem {
                                     // acquires this barrier), and the commit of S[b]
   uint64_t p_full[2];               // P~[b] written by all 8 softmax warps; this also
                                     // says S[b] was read and inner[b] of tile t-2 folded
-  uint64_t i_full[2];               // inner[b] written (tcgen05.commit)
+  uint64_t i_full[2];               // two arrivals: the MMA thread after it saw p_full (so
+                                    // alpha of the tile is visible), and the commit of inner[b]
+  uint64_t i_empty[2];              // the correction warpgroup read inner[b]
+  uint64_t l_full;                  // the softmax warps published the row sums
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -166,38 +171,39 @@ __device__ __forceinline__ float exp_pack_store(const float (&x)[32], float2 L2,
   return s2.x + s2.y;
 }
 
-// acc = alpha * acc + inner (the outer level of the accumulation) for the
-// thread's two rows (alpha.x row r0, alpha.y row r0+8), reading inner from
-// TMEM at taddr with .16x256b loads (layout of acc: see the softmax role).
-template <int D>
-__device__ __forceinline__ void fold_inner(float (&acc)[D / 2], uint32_t taddr, float2 alpha) {
-  const float2 a0 = make_float2(alpha.x, alpha.x), a1 = make_float2(alpha.y, alpha.y);
-  uint32_t in[D / 2];
-  tmem_ld16x256_32(taddr, *reinterpret_cast<uint32_t(*)[32]>(in));
-  if (D == 128) tmem_ld16x256_32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(in + (D == 128 ? 32 : 0)));
-  tmem_ld_wait();
+// acc[32 channels] = alpha * acc + inner for one row (.32x32b load).
+__device__ __forceinline__ void fold32(float* acc, const uint32_t (&in)[32], float al) {
+  const float2 al2 = make_float2(al, al);
 #pragma unroll
-  for (int i = 0; i < D / 2; i += 4) {
-    const float2 r0 = __ffma2_rn(a0, make_float2(acc[i], acc[i + 1]),
-                                 make_float2(__uint_as_float(in[i]), __uint_as_float(in[i + 1])));
-    const float2 r1 = __ffma2_rn(a1, make_float2(acc[i + 2], acc[i + 3]),
-                                 make_float2(__uint_as_float(in[i + 2]), __uint_as_float(in[i + 3])));
-    acc[i] = r0.x;
-    acc[i + 1] = r0.y;
-    acc[i + 2] = r1.x;
-    acc[i + 3] = r1.y;
+  for (int c = 0; c < 32; c += 2) {
+    const float2 r = __ffma2_rn(al2, make_float2(acc[c], acc[c + 1]),
+                                make_float2(__uint_as_float(in[c]), __uint_as_float(in[c + 1])));
+    acc[c] = r.x;
+    acc[c + 1] = r.y;
   }
 }
 
-// Two adjacent output channels (index of the first, even) in the output type.
+// Eight consecutive output channels (index of the first, a multiple of 8) in
+// the output type, with 16-byte stores.
 template <int OT>
-__device__ __forceinline__ void store_pair(void* out, size_t idx, float f0, float f1) {
+__device__ __forceinline__ void store8(void* out, size_t idx, const float (&f)[8]) {
   if (OT == 2) {
-    *reinterpret_cast<float2*>(static_cast<float*>(out) + idx) = make_float2(f0, f1);
-  } else if (OT == 0) {
-    *reinterpret_cast<__half2*>(static_cast<uint16_t*>(out) + idx) = __floats2half2_rn(f0, f1);
+    float4* p = reinterpret_cast<float4*>(static_cast<float*>(out) + idx);
+    p[0] = make_float4(f[0], f[1], f[2], f[3]);
+    p[1] = make_float4(f[4], f[5], f[6], f[7]);
   } else {
-    *reinterpret_cast<__nv_bfloat162*>(static_cast<uint16_t*>(out) + idx) = __floats2bfloat162_rn(f0, f1);
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (OT == 0) {
+        const __half2 hv = __floats2half2_rn(f[2 * u], f[2 * u + 1]);
+        w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+      } else {
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(f[2 * u], f[2 * u + 1]);
+        w[u] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+    }
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + idx) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -228,9 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 2);
       mbar_init(&sm.p_full[b], 8);
-      mbar_init(&sm.i_full[b], 1);
+      mbar_init(&sm.i_full[b], 2);
+      mbar_init(&sm.i_empty[b], 4);
     }
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.l_full, 8);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -307,8 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int u) -> bool {
         const int s = u % kStages, b = u & 1;
-        // P~(u) is written; inner[b] was folded (tile u-2) before that arrive
+        // P~(u) and alpha(u) are written; the correction warpgroup has read
+        // inner[b] of tile u-2
         if (!mbar_wait(&sm.p_full[b], (u >> 1) & 1, abort_flag)) return false;
+        if (u >= 2 && !mbar_wait(&sm.i_empty[b], ((u >> 1) - 1) & 1, abort_flag)) return false;
+        mbar_arrive(&sm.i_full[b]);                       // releases the p_full acquire (alpha)
         tc_fence_after();
         const uint64_t pb = dp + b * kStageP, vb = dv + s * kStageV;
 #pragma unroll
@@ -331,19 +342,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sm.drain, 0, nullptr);
       }
     }
-  } else if (wg >= 1) {
+  } else if (wg == 1 || wg == 2) {
     // ------------------------------------------------------------ softmax warpgroups
     // Raised inside the branch it governs, so that the compiler allocates this
-    // role's code against the larger budget (40*128 + 232*256 <= 168*384).
-    setmaxnreg_inc<232>();
+    // role's code against the larger budget (40*128 + 152*256 + 168*128 = 128*512).
+    setmaxnreg_inc<152>();
     // The .16x256b TMEM loads give thread t of a warp, in a 16-lane group, the
     // two lanes t/4 and t/4 + 8 and the columns 8k + 2g + {0,1} (g = t%4,
     // k = 0..15).  Warpgroup h takes lanes 16h..16h+15 of each 32-lane
     // quadrant, so every query row is shared by the four threads g = 0..3 of
     // one warp and each thread owns two rows.  With the K^ rows of each block
     // stored so that column 8k + 2g + e holds token 32g + 2k + e, thread g sees
-    // the 32 consecutive keys 32g..32g+31 of the tile (both rows), and the
-    // inner-product columns it loads are output channels 8k + 2g + {0,1}.
+    // the 32 consecutive keys 32g..32g+31 of the tile (both rows).
     const int h = wg - 1;
     const int quad = warp & 3;
     const int g = lane & 3;
@@ -351,17 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row0 = qt * 128 + r0, row1 = row0 + 8;      // rows in the head
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quad + 16 * h) << 16;
     const uint32_t tS = tmem + lane_addr;                 // + 128*b: S buffer b
-    const uint32_t tI = tmem + lane_addr + 256;           // + D*b: inner buffer b
-    for (int i = threadIdx.x - 128 * wg; i < D; i += 128)
-      sm.vsc[h][i] = v_scale[static_cast<size_t>(bh) * D + i];
-    named_bar_sync(1 + h, 128);
-    // acc[4k + e] / acc[4k + 2 + e]: rows r0 / r0+8, channel 8k + 2g + e
-    // (k < 8; channels 64 + ... in the second half when D = 128)
-    float acc[D / 2];
-#pragma unroll
-    for (int c = 0; c < D / 2; ++c) acc[c] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float2 al_1 = make_float2(0.f, 0.f), al_2 = make_float2(0.f, 0.f);  // (row0, row1) alpha of tiles t-1, t-2
     bool ok = mbar_wait_warp(&sm.q_full, 0, abort_flag);
     const float a0 = ok ? sm.qsc[r0] : 0.f, a1 = ok ? sm.qsc[r0 + 8] : 0.f;
     const float2 a02 = make_float2(a0, a0), a12 = make_float2(a1, a1);
@@ -377,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < nt; ++t) {
       const int s = t % kStages, b = t & 1;
       // s_full(t) also says PV(t-2) is complete: the MMA thread issued QK(t)
-      // after PV(t-2), and the commit tracks every earlier MMA.  So inner(t-2)
-      // can be folded now and P~[b] is free, with no wait of their own.
+      // after PV(t-2), and the commit tracks every earlier MMA.  So P~[b] is
+      // free, with no wait of its own.
       if (ok) ok = mbar_wait_warp(&sm.s_full[b], (t >> 1) & 1, abort_flag);
       if (!ok) {
         if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
@@ -386,7 +386,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       tc_fence_after();
-      if (t >= 2) fold_inner<D>(acc, tI + b * D, al_2);   // outer level for tile t-2
       float x0[32], x1[32];                               // rows r0, r0+8; keys 32g + j
       {
         uint32_t sA[32], sB[32];
@@ -415,6 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
       const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
       const float2 alpha = make_float2(ex2((m0 - mn0) * L), ex2((m1 - mn1) * L));  // 0 on the first tile
+      // for the correction warpgroup; slot t%4 was last read for tile t-4,
+      // before PV(t-2) was issued, which s_full(t) follows
+      if (g == 0) {
+        sm.alpha[t & 3][r0] = alpha.x;
+        sm.alpha[t & 3][r0 + 8] = alpha.y;
+      }
       // p448 = 448 * exp2((x' - m) L) = exp2(x' L - (m L - log2 448))
       const float2 nb0 = make_float2(kLog2_448 - mn0 * L, kLog2_448 - mn0 * L);
       const float2 nb1 = make_float2(kLog2_448 - mn1 * L, kLog2_448 - mn1 * L);
@@ -428,48 +433,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float s1 = exp_pack_store(x1, L2, nb1, p1, g, r0 & 7);
       named_bar_arrive(bar_other, 64);
       fence_proxy_async_smem();
-      tc_fence_before();                                  // S(t) and inner(t-2) reads are done
+      tc_fence_before();                                  // S(t) reads are done
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[b]);
       l0 = alpha.x * l0 + s0;
       l1 = alpha.y * l1 + s1;
       m0 = mn0;
       m1 = mn1;
-      al_2 = al_1;
-      al_1 = alpha;
     }
     // the second warpgroup's last turn ended
     if (h == 0 && nt > 0) named_bar_sync(bar_mine, 64);
-    if (ok) {
-      // the last one or two inner products: i_full of the last tile's PV covers
-      // every MMA issued before it
-      const int u = nt - 1, ub = u & 1;
-      ok = mbar_wait_warp(&sm.i_full[ub], (u >> 1) & 1, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        if (nt >= 2) fold_inner<D>(acc, tI + (ub ^ 1) * D, al_2);
-        fold_inner<D>(acc, tI + ub * D, al_1);
-      }
-    }
     if (ok) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      const float inv0 = 1.0f / l0, inv1 = 1.0f / l1;
-      const float* vs = sm.vsc[h];
+      if (g == 0) {
+        sm.lsum[r0] = l0;
+        sm.lsum[r0 + 8] = l1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.l_full);
+    }
+  } else if (wg == 3) {
+    // ------------------------------------------------------------ correction warpgroup
+    // Thread r owns query row r (TMEM lane r, .32x32b loads: consecutive
+    // channels) and the outer fp32 accumulator of the two-level accumulation
+    // in registers: per key tile, acc = alpha*acc + inner (inner = the fresh
+    // PV accumulator of that tile), then the epilogue O = acc*v_scale/l.
+    setmaxnreg_inc<168>();
+    const int r = (warp & 3) * 32 + lane;
+    const int row = qt * 128 + r;
+    const uint32_t tI = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + 256;
+    for (int i = r; i < D; i += 128) sm.vsc[i] = v_scale[static_cast<size_t>(bh) * D + i];
+    named_bar_sync(1, 128);
+    float acc[D];
 #pragma unroll
-      for (int i = 0; i < D / 2; i += 4) {
-        const int c = 8 * ((i >> 2) & 7) + 2 * g + 64 * (i >> 5);   // channel of acc[i], acc[i+1]
-        const float v0 = vs[c], v1 = vs[c + 1];
-        if (row0 < N) store_pair<OT>(out, (static_cast<size_t>(bh) * N + row0) * D + c,
-                                     acc[i] * v0 * inv0, acc[i + 1] * v1 * inv0);
-        if (row1 < N) store_pair<OT>(out, (static_cast<size_t>(bh) * N + row1) * D + c,
-                                     acc[i + 2] * v0 * inv1, acc[i + 3] * v1 * inv1);
+    for (int c = 0; c < D; ++c) acc[c] = 0.f;
+    bool ok = true;
+    for (int t = 0; ok && t < nt; ++t) {
+      const int b = t & 1;
+      // i_full also carries the MMA thread's release after it saw p_full, so
+      // alpha of tile t is visible
+      if (!mbar_wait_warp(&sm.i_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const float al = sm.alpha[t & 3][r];
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tI + b * D + c0, v);
+        tmem_ld_wait();
+        fold32(acc + c0, v, al);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.i_empty[b]);
+    }
+    if (ok) ok = mbar_wait_warp(&sm.l_full, 0, abort_flag);
+    if (ok && row < N) {
+      const float inv = 1.0f / sm.lsum[r];
+      const size_t obase = (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 8) {
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] = acc[c + u] * sm.vsc[c + u] * inv;
+        store8<OT>(out, obase + c, f);
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
