@@ -416,10 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 alpha = make_float2(ex2((m0 - mn0) * L), ex2((m1 - mn1) * L));  // 0 on the first tile
       // for the correction warpgroup; slot t%4 was last read for tile t-4,
       // before PV(t-2) was issued, which s_full(t) follows
-      if (g == 0) {
-        sm.alpha[t & 3][r0] = alpha.x;
-        sm.alpha[t & 3][r0 + 8] = alpha.y;
-      }
+      sm.alpha[t & 3][r0] = alpha.x;                      // the row's four threads agree
+      sm.alpha[t & 3][r0 + 8] = alpha.y;
       // p448 = 448 * exp2((x' - m) L) = exp2(x' L - (m L - log2 448))
       const float2 nb0 = make_float2(kLog2_448 - mn0 * L, kLog2_448 - mn0 * L);
       const float2 nb1 = make_float2(kLog2_448 - mn1 * L, kLog2_448 - mn1 * L);
@@ -435,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();                                  // S(t) reads are done
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[b]);
+      mbar_arrive_lane0(&sm.p_full[b], lane);
       l0 = alpha.x * l0 + s0;
       l1 = alpha.y * l1 + s1;
       m0 = mn0;
@@ -448,12 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      if (g == 0) {
-        sm.lsum[r0] = l0;
-        sm.lsum[r0 + 8] = l1;
-      }
+      sm.lsum[r0] = l0;                                   // the row's four threads agree
+      sm.lsum[r0 + 8] = l1;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.l_full);
+      mbar_arrive_lane0(&sm.l_full, lane);
     }
   } else if (wg == 3) {
     // ------------------------------------------------------------ correction warpgroup
@@ -487,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.i_empty[b]);
+      mbar_arrive_lane0(&sm.i_empty[b], lane);
     }
     if (ok) ok = mbar_wait_warp(&sm.l_full, 0, abort_flag);
     if (ok && row < N) {
