@@ -4,7 +4,7 @@
 // Per-thread INT4 Quantization" (arxiv.science abstract page, Abstract): the
 // INT4 Q^K^T product, FP8 P~ and V, and the two-level accumulation of P~V.
 //
-// One CTA = one 128-row query block of one head; 384 threads, warp-specialised:
+// One CTA = one 128-row query block of one head; 512 threads, warp-specialised:
 //   warp 0        TMA producer: the Q^ tile once, then per key tile K^, V^T,
 //                 the key scales and the correction chunk (kStages-deep ring).
 //   warp 1        MMA issuer (one thread): S = Q^ K^T with tcgen05 kind::f8f6f4
@@ -16,12 +16,15 @@
 //   warps 4-7,    two softmax warpgroups.  Warpgroup h owns lanes 16h..16h+15 of
 //   warps 8-11    every 32-lane TMEM quadrant; with .16x256b loads a thread owns
 //                 two query rows and 32 consecutive keys of each tile (four
-//                 threads of a warp share a row).  Per tile: fold the inner
-//                 product of tile t-2 into the register accumulator (acc =
-//                 alpha*acc + inner: the outer level of the two-level
-//                 accumulation), dequantise + correct its 64 scores, row max
-//                 across the four threads, exp2, l, and P~ = e4m3(448 p) into
-//                 shared memory (the MMA's swizzled layout).
+//                 threads of a warp share a row).  Per tile: dequantise +
+//                 correct its 64 scores, row max across the four threads, the
+//                 rescale factor alpha (to shared memory), exp2, l, and
+//                 P~ = e4m3(448 p) into shared memory (the MMA's swizzled
+//                 layout).  The exp2 phases of the two warps of a sub-partition
+//                 take turns (named barriers).
+//   warps 12-15   correction warpgroup: thread r owns query row r and the outer
+//                 fp32 accumulator (acc = alpha*acc + inner per key tile: the
+//                 outer level of the two-level accumulation), then the epilogue.
 // TMEM columns: S[b] at 128*b (b = 0, 1), inner[b] at 256 + d*b.
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout the kernel
 // records it in the device error word and every role leaves its loop.
