@@ -29,6 +29,17 @@ constants and in the function docstrings):
                        (outer level).
   7. attn_fp64         the unquantized reference  softmax(QK^T * sm_scale) V.
 
+Two variants beyond the abstract's method, both readings fixed before any
+kernel was written:
+  - INT8 Q/K (quant_int8_rows): the predecessor's 8-bit integer quantization
+    ("SageAttention: Accurate 8-Bit Attention", ainnect.com/research/19
+    summary) on [-127, 127], one scale per token, with everything else of the
+    path unchanged (smoothing, correction, FP8 P~V, two-level accumulation).
+  - V smoothing (token_mean, quant_v_smoothed): subtract the per-channel token
+    mean of V before FP8 and add it back to O ("smooth V" in the SageAttention2
+    summary, ainnect.com/research/55).  The softmax weights of a row sum to one,
+    so sum_j p_j (V_j - vbar) / l + vbar is the same attention output.
+
 Precision.  Steps 1-3 and 5 produce the payloads (the integers, codes and
 scales the kernels also produce); they are written in float32 with a fixed
 operation order so that they are reproducible bit for bit.  Steps 4, 6 and 7
@@ -50,6 +61,7 @@ import numpy as np
 BM = 128            # rows of Q per smoothing block / per attention tile
 BN = 128            # keys per attention tile (the "inner" accumulation block)
 INT4_MAX = 7        # symmetric INT4 range [-7, 7]
+INT8_MAX = 127      # symmetric INT8 range [-127, 127] (the INT8 variant)
 E4M3_MAX = 448.0    # largest finite e4m3 value; also the fixed P~ scale
 LOG2E = 1.4426950408889634
 
@@ -197,10 +209,31 @@ def quant_int4_rows(X: np.ndarray):
     return q, scale
 
 
-def smooth_quant_qk(Q: np.ndarray, K: np.ndarray):
+def quant_int8_rows(X: np.ndarray):
+    """The INT8 variant: X [n, d] float32 -> (q int8 [n, d], scale float32 [n]).
+    scale = amax/127 and inv = 127/amax (float32 IEEE), q = RNE(x*inv)
+    clamped to [-127, 127]; an all-zero row gets scale 0 and q = 0."""
+    X = np.asarray(X, np.float32)
+    amax = np.max(np.abs(X), axis=1)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    scale = np.where(nz, safe / np.float32(INT8_MAX), np.float32(0)).astype(np.float32)
+    inv = (np.float32(INT8_MAX) / safe).astype(np.float32)
+    y = (X * inv[:, None]).astype(np.float32)
+    q = np.clip(np.rint(y), -INT8_MAX, INT8_MAX).astype(np.int8)
+    q[~nz] = 0
+    return q, scale
+
+
+def smooth_quant_qk(Q: np.ndarray, K: np.ndarray, qk_bits: int = 4):
     """One head. Q, K: [N, d]. Returns the padded payloads:
     q_i4 [Np, d] int8, q_scale [Np] f32, q_mean [Np/BM, d] f32,
-    k_i4 [Np, d] int8, k_scale [Np] f32, k_mean [d] f32.  Rows >= N are 0."""
+    k_i4 [Np, d] int8, k_scale [Np] f32, k_mean [d] f32.  Rows >= N are 0.
+    qk_bits = 4 (the method: INT4 values) or 8 (the INT8 variant; the integer
+    payloads then hold values in [-127, 127] under the same keys)."""
+    if qk_bits not in (4, 8):
+        raise ValueError("qk_bits must be 4 or 8")
+    quant = quant_int4_rows if qk_bits == 4 else quant_int8_rows
     Q = np.asarray(Q, np.float32)
     K = np.asarray(K, np.float32)
     N, d = Q.shape
@@ -213,8 +246,8 @@ def smooth_quant_qk(Q: np.ndarray, K: np.ndarray):
     k_i4 = np.zeros((Np, d), np.int8)
     q_scale = np.zeros(Np, np.float32)
     k_scale = np.zeros(Np, np.float32)
-    q_i4[:N], q_scale[:N] = quant_int4_rows(Qs)
-    k_i4[:N], k_scale[:N] = quant_int4_rows(Ks)
+    q_i4[:N], q_scale[:N] = quant(Qs)
+    k_i4[:N], k_scale[:N] = quant(Ks)
     return dict(q_i4=q_i4, q_scale=q_scale, q_mean=qbar, k_i4=k_i4,
                 k_scale=k_scale, k_mean=kbar)
 
@@ -259,13 +292,28 @@ def quant_v(V: np.ndarray):
     return vt, sv
 
 
+def token_mean(V: np.ndarray) -> np.ndarray:
+    """V smoothing's per-channel mean: the same fixed-order float32 token mean
+    as k_mean (128-token chunks, chunk sums in order, one division by N)."""
+    return k_mean(V)
+
+
+def quant_v_smoothed(V: np.ndarray):
+    """The V-smoothing variant: vbar = token_mean(V), then quant_v of
+    V - vbar (float32).  Returns (v_t codes [d, Np], v_scale [d], vbar [d])."""
+    V = np.asarray(V, np.float32)
+    vbar = token_mean(V)
+    vt, sv = quant_v((V - vbar[None, :]).astype(np.float32))
+    return vt, sv, vbar
+
+
 # ----------------------------------------------------------------------------
 # Step 6 - attention over the quantized payloads.
 # ----------------------------------------------------------------------------
 
 def qk_int(q_i4: np.ndarray, k_i4: np.ndarray) -> np.ndarray:
-    """Exact integer Q^ K^T (int64): the INT4 matrix product."""
-    # fp64 matmul of small integers is exact (|sum| <= 49*d << 2^53)
+    """Exact integer Q^ K^T (int64): the INT4 (or INT8-variant) matrix product."""
+    # fp64 matmul of small integers is exact (|sum| <= 127^2*d << 2^53)
     return (np.asarray(q_i4, np.float64) @ np.asarray(k_i4, np.float64).T).astype(np.int64)
 
 
@@ -287,8 +335,9 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
         P~   = e4m3(448 p)
         inner= P~ . V~  over this tile only              (inner level)
         acc  = alpha*acc + inner                          (outer level)
-    then O = acc * sv / (448 l).  'amb' bounds what a different but equally
-    correct rounding of ambiguous 448p values (see AMBIG_REL) can change.
+    then O = acc * sv / (448 l), plus p['v_mean'] when V was smoothed.
+    'amb' bounds what a different but equally correct rounding of ambiguous
+    448p values (see AMBIG_REL) can change.
     """
     Np = n_pad(N)
     nb = Np // BM
@@ -308,6 +357,7 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
         sv = np.ones(vdec.shape[1])
     C = np.asarray(p["C"], np.float64)
     d = vdec.shape[1]
+    vbar = np.asarray(p["v_mean"], np.float64) if p.get("v_mean") is not None else np.zeros(d)
     blocks = range(nb) if q_blocks is None else q_blocks
     outs, ambs, rows = [], [], []
     for b in blocks:
@@ -341,7 +391,7 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
             amb = alpha[:, None] * amb + gap @ np.abs(vdec[c])
             m = m_new
         scale = E4M3_MAX if quantize else 1.0
-        outs.append(acc * sv[None, :] / (scale * l[:, None]))
+        outs.append(acc * sv[None, :] / (scale * l[:, None]) + vbar[None, :])
         ambs.append(amb * sv[None, :] / (scale * l[:, None]))
         rows.append(r)
     if not outs:
@@ -372,17 +422,22 @@ def attn_fp64(Q, K, V, causal: bool, sm_scale: float, rows=None) -> np.ndarray:
 # The whole pipeline for one head.
 # ----------------------------------------------------------------------------
 
-def sage2_head(Q, K, V, causal: bool, sm_scale: float | None = None, q_blocks=None):
+def sage2_head(Q, K, V, causal: bool, sm_scale: float | None = None, q_blocks=None,
+               qk_bits: int = 4, smooth_v: bool = False):
     """Steps 1-6 for one head.  Q, K, V: [N, d] (fp16/bf16 values as float32).
-    Returns (payload dict, O rows, amb rows, row index)."""
+    qk_bits 4 (the method) or 8 (the INT8 variant); smooth_v selects the V
+    smoothing variant.  Returns (payload dict, O rows, amb rows, row index)."""
     Q = np.asarray(Q, np.float32)
     K = np.asarray(K, np.float32)
     V = np.asarray(V, np.float32)
     N, d = Q.shape
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
-    pay = smooth_quant_qk(Q, K)
+    pay = smooth_quant_qk(Q, K, qk_bits)
     pay["C"] = qk_correction(pay["q_mean"], K)
-    pay["v_t"], pay["v_scale"] = quant_v(V)
+    if smooth_v:
+        pay["v_t"], pay["v_scale"], pay["v_mean"] = quant_v_smoothed(V)
+    else:
+        pay["v_t"], pay["v_scale"] = quant_v(V)
     O, amb, rows = attn_quantized(pay, N, causal, sm_scale, q_blocks=q_blocks)
     return pay, O, amb, rows
