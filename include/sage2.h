@@ -68,6 +68,17 @@ typedef enum {
 typedef enum { SAGE2_F16 = 0, SAGE2_BF16 = 1, SAGE2_F32 = 2 } sage2_dtype;
 
 /*
+ * Integer format of the Q^/K^ payloads (q_i4, k_i4).
+ *   SAGE2_QK_INT4 : the method.  Values in [-7,7], each stored as its e4m3 code.
+ *   SAGE2_QK_INT8 : a variant, the 8-bit quantization of the predecessor
+ *                   ("SageAttention: Accurate 8-Bit Attention", ainnect.com
+ *                   research/19 summary).  Values in [-127,127] stored as
+ *                   two's-complement bytes; scale = amax/127.  Everything else on
+ *                   the path is unchanged (smoothing, correction, FP8 P~V).
+ */
+typedef enum { SAGE2_QK_INT4 = 0, SAGE2_QK_INT8 = 1 } sage2_qk_format;
+
+/*
  * Smoothing + INT4 quantization of Q and K, and the Q-smoothing correction.
  * (Abstract: INT4 (Q,K) at per-thread granularity; "a method to smooth Q".)
  *   q, k      : [B,H,N,d] in `dtype` (SAGE2_F16 or SAGE2_BF16).
@@ -85,6 +96,14 @@ sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int 
                                    uint8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
                                    sage2_stream_t stream);
 
+/* As sage2_smooth_quant_qk with the payload format chosen by `qk_format`
+ * (sage2_qk_format; SAGE2_ERR_INVALID_ARG otherwise).  INT8: scale = amax/127,
+ * q = clamp(rint(x * (127/amax)), -127, 127) as int8 bytes. */
+sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, int B, int H, int N,
+                                      int d, uint8_t* q_i4, float* q_scale, float* q_mean,
+                                      uint8_t* k_i4, float* k_scale, float* k_mean,
+                                      float* qk_corr, int qk_format, sage2_stream_t stream);
+
 /*
  * FP8 e4m3 quantization of V with one scale per channel (Abstract: FP8 V).
  *   v        : [B,H,N,d] in `dtype`.
@@ -94,6 +113,17 @@ sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int 
  */
 sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d,
                            uint8_t* v_fp8_t, float* v_scale, sage2_stream_t stream);
+
+/*
+ * As sage2_quant_v, with V smoothing when v_mean is not NULL ("smooth V",
+ * ainnect.com/research/55 summary of SageAttention2): v_mean [B,H,d] receives
+ * the per-channel token mean of V (the fixed fp32 order of the K mean), and the
+ * codes and scales are those of fp32(V) - v_mean.  The attention adds v_mean
+ * back to O (sage2_attn_fwd_quantized_ex).  v_mean must be 16-byte aligned.
+ */
+sage2_status sage2_quant_v_ex(const void* v, int dtype, int B, int H, int N, int d,
+                              uint8_t* v_fp8_t, float* v_scale, float* v_mean,
+                              sage2_stream_t stream);
 
 /*
  * Attention over the quantized payloads (the fused tcgen05 kernel alone).
@@ -113,6 +143,16 @@ sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
                                       int N, int d, int causal, float sm_scale,
                                       sage2_stream_t stream);
 
+/* As sage2_attn_fwd_quantized for payloads in `qk_format`, and with
+ * O = acc*v_scale/(448 l) + v_mean when v_mean is not NULL (V smoothed by
+ * sage2_quant_v_ex). */
+sage2_status sage2_attn_fwd_quantized_ex(const uint8_t* q_i4, const float* q_scale,
+                                         const uint8_t* k_i4, const float* k_scale,
+                                         const float* qk_corr, const uint8_t* v_fp8_t,
+                                         const float* v_scale, const float* v_mean, void* o,
+                                         int o_dtype, int B, int H, int N, int d, int causal,
+                                         float sm_scale, int qk_format, sage2_stream_t stream);
+
 /*
  * The whole forward pass: smoothing + quantization of Q, K, V, the correction
  * and the attention kernel, with the payloads in a workspace that the library
@@ -124,6 +164,14 @@ sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
 sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
                             int N, int d, int dtype, int o_dtype, int causal, float sm_scale,
                             sage2_stream_t stream);
+
+/* The whole forward pass with the variants: qk_format (sage2_qk_format) and
+ * smooth_v (0 or 1: V smoothing, see sage2_quant_v_ex).  sage2_attn_fwd is
+ * this call with SAGE2_QK_INT4 and smooth_v = 0. */
+sage2_status sage2_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, int B,
+                               int H, int N, int d, int dtype, int o_dtype, int causal,
+                               float sm_scale, int qk_format, int smooth_v,
+                               sage2_stream_t stream);
 
 /*
  * The same forward pass as sage2_attn_fwd, for callers that must not have the
@@ -158,6 +206,11 @@ size_t sage2_workspace_bytes(int B, int H, int N, int d);
  */
 sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
                                 int d, int32_t* s_out, sage2_stream_t stream);
+
+/* As sage2_debug_qk_s32 for payloads in `qk_format`; INT8 payloads go through
+ * the attention kernel's 8-bit integer path (tcgen05 kind::i8, s32). */
+sage2_status sage2_debug_qk_s32_ex(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
+                                   int d, int qk_format, int32_t* s_out, sage2_stream_t stream);
 
 /*
  * Synchronizes `stream`, then reads and clears the device error word that

@@ -25,6 +25,8 @@ __all__ = [
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage2.so")
 F16, BF16, F32 = 0, 1, 2
+QK_INT4, QK_INT8 = 0, 1
+_QKF = {4: QK_INT4, 8: QK_INT8}
 _DT = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
 STATUS = {0: "SAGE2_OK", 1: "SAGE2_ERR_INVALID_ARG", 2: "SAGE2_ERR_UNSUPPORTED",
           3: "SAGE2_ERR_MISALIGNED", 4: "SAGE2_ERR_CUDA", 5: "SAGE2_ERR_NO_MEM",
@@ -42,6 +44,12 @@ _SIGS = {
     "sage2_attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage2_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "sage2_debug_qk_s32": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
+    "sage2_smooth_quant_qk_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "sage2_quant_v_ex": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "sage2_attn_fwd_quantized_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                         _F, _I, _P]),
+    "sage2_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "sage2_debug_qk_s32_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "sage2_check_device_error": (_I, [_P]),
     "sage2_status_string": (ctypes.c_char_p, [_I]),
     "sage2_version": (_I, []),
@@ -118,10 +126,20 @@ def sage2_check_device_error(device=None) -> int:
     return int(lib().sage2_check_device_error(st))
 
 
-def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = None) -> dict:
-    """Smoothing + INT4 of Q and K and the Q-smoothing correction.
-    Returns the payload dict (q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
-    `out`, if given, is such a dict (from an earlier call) and is overwritten."""
+def _qk_bits_of(t: torch.Tensor) -> int:
+    """Payload format from the payload dtype: uint8 e4m3 codes (INT4), int8 (INT8)."""
+    return 8 if t.dtype == torch.int8 else 4
+
+
+def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = None,
+                          qk_bits: int = 4) -> dict:
+    """Smoothing + INT4 (qk_bits=4, the method) or INT8 (qk_bits=8, the variant)
+    of Q and K and the Q-smoothing correction.  Returns the payload dict (q_i4,
+    q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr); q_i4/k_i4 are uint8 e4m3
+    codes for INT4 and int8 values for INT8.  `out`, if given, is such a dict
+    (from an earlier call with the same qk_bits) and is overwritten."""
+    if qk_bits not in _QKF:
+        raise ValueError("qk_bits must be 4 or 8")
     B, H, N, d = _dims(q)
     if k.shape != q.shape or k.dtype != q.dtype:
         raise ValueError("q and k must have the same shape and dtype")
@@ -130,62 +148,77 @@ def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = N
     NB = Np // 128
     dev = q.device
     if out is None:
-        out = _qk_payloads(B, H, Np, NB, d, dev)
-    st = lib().sage2_smooth_quant_qk(
+        out = _qk_payloads(B, H, Np, NB, d, dev, qk_bits)
+    elif _qk_bits_of(out["q_i4"]) != qk_bits:
+        raise ValueError("out holds payloads of the other qk_bits")
+    st = lib().sage2_smooth_quant_qk_ex(
         _ptr(q), _ptr(k), _DT[q.dtype], B, H, N, d, _ptr(out["q_i4"]), _ptr(out["q_scale"]),
         _ptr(out["q_mean"]), _ptr(out["k_i4"]), _ptr(out["k_scale"]), _ptr(out["k_mean"]),
-        _ptr(out["qk_corr"]), _stream(q))
-    _check("sage2_smooth_quant_qk", st)
+        _ptr(out["qk_corr"]), _QKF[qk_bits], _stream(q))
+    _check("sage2_smooth_quant_qk_ex", st)
     return out
 
 
-def _qk_payloads(B, H, Np, NB, d, dev) -> dict:
+def _qk_payloads(B, H, Np, NB, d, dev, qk_bits=4) -> dict:
+    ity = torch.uint8 if qk_bits == 4 else torch.int8   # e4m3 codes of INT4 values / INT8 values
     return dict(
-        q_i4=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),   # e4m3 codes of INT4 values
+        q_i4=torch.empty(B, H, Np, d, dtype=ity, device=dev),
         q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
         q_mean=torch.empty(B, H, NB, d, dtype=torch.float32, device=dev),
-        k_i4=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),   # e4m3 codes, rows permuted per block
+        k_i4=torch.empty(B, H, Np, d, dtype=ity, device=dev),   # rows permuted per block
         k_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
         k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev),
         qk_corr=torch.empty(B, H, NB, Np, dtype=torch.float32, device=dev),
     )
 
 
-def sage2_quant_v(v: torch.Tensor, out: tuple | None = None):
-    """FP8 e4m3 V per channel. Returns (v_fp8_t uint8 [B,H,d,Np], v_scale f32 [B,H,d]);
-    `out`, if given, is such a pair (from an earlier call) and is overwritten."""
+def sage2_quant_v(v: torch.Tensor, out: tuple | None = None, smooth: bool = False):
+    """FP8 e4m3 V per channel. Returns (v_fp8_t uint8 [B,H,d,Np], v_scale f32 [B,H,d]),
+    and with smooth=True (V smoothing) also v_mean f32 [B,H,d]; `out`, if given,
+    is such a tuple (from an earlier call) and is overwritten."""
     B, H, N, d = _dims(v)
     Np = n_pad(N)
     if out is None:
         vt = torch.empty(B, H, d, Np, dtype=torch.uint8, device=v.device)
         vs = torch.empty(B, H, d, dtype=torch.float32, device=v.device)
+        vm = torch.empty(B, H, d, dtype=torch.float32, device=v.device) if smooth else None
     else:
-        vt, vs = out
-    st = lib().sage2_quant_v(_ptr(v), _DT[v.dtype], B, H, N, d, _ptr(vt), _ptr(vs), _stream(v))
-    _check("sage2_quant_v", st)
-    return vt, vs
+        vt, vs = out[0], out[1]
+        vm = out[2] if smooth else None
+    st = lib().sage2_quant_v_ex(_ptr(v), _DT[v.dtype], B, H, N, d, _ptr(vt), _ptr(vs), _ptr(vm),
+                                _stream(v))
+    _check("sage2_quant_v_ex", st)
+    return (vt, vs, vm) if smooth else (vt, vs)
 
 
 def sage2_attn_fwd_quantized(pay: dict, v_fp8_t: torch.Tensor, v_scale: torch.Tensor, N: int,
                              causal: bool, sm_scale: float, out_dtype=torch.float32,
-                             out: torch.Tensor | None = None) -> torch.Tensor:
+                             out: torch.Tensor | None = None,
+                             v_mean: torch.Tensor | None = None) -> torch.Tensor:
     """The attention kernel alone, over payloads from sage2_smooth_quant_qk /
-    sage2_quant_v (or any tensors in those layouts)."""
+    sage2_quant_v (or any tensors in those layouts).  The payload format (INT4 or
+    INT8) follows the q_i4 dtype; v_mean is the token mean of a smoothed V."""
     B, H, Np, d = pay["q_i4"].shape
     if out is None:
         out = torch.empty(B, H, N, d, dtype=out_dtype, device=pay["q_i4"].device)
-    st = lib().sage2_attn_fwd_quantized(
+    st = lib().sage2_attn_fwd_quantized_ex(
         _ptr(pay["q_i4"]), _ptr(pay["q_scale"]), _ptr(pay["k_i4"]), _ptr(pay["k_scale"]),
-        _ptr(pay["qk_corr"]), _ptr(v_fp8_t), _ptr(v_scale), _ptr(out), _DT[out.dtype],
-        B, H, N, d, int(bool(causal)), float(sm_scale), _stream(out))
-    _check("sage2_attn_fwd_quantized", st)
+        _ptr(pay["qk_corr"]), _ptr(v_fp8_t), _ptr(v_scale), _ptr(v_mean), _ptr(out),
+        _DT[out.dtype], B, H, N, d, int(bool(causal)), float(sm_scale),
+        _QKF[_qk_bits_of(pay["q_i4"])], _stream(out))
+    _check("sage2_attn_fwd_quantized_ex", st)
     return out
 
 
 def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                    sm_scale: float | None = None, out_dtype=None,
-                   out: torch.Tensor | None = None) -> torch.Tensor:
-    """Full forward pass (quantization + correction + attention) on q's stream."""
+                   out: torch.Tensor | None = None, qk_bits: int = 4,
+                   smooth_v: bool = False) -> torch.Tensor:
+    """Full forward pass (quantization + correction + attention) on q's stream.
+    qk_bits 4 is the method (INT4 Q/K); 8 is the INT8 variant.  smooth_v turns
+    on V smoothing."""
+    if qk_bits not in _QKF:
+        raise ValueError("qk_bits must be 4 or 8")
     B, H, N, d = _dims(q)
     for t in (k, v):
         if t.shape != q.shape or t.dtype != q.dtype:
@@ -195,9 +228,10 @@ def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bo
         sm_scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty(B, H, N, d, dtype=out_dtype or q.dtype, device=q.device)
-    st = lib().sage2_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, _DT[q.dtype],
-                              _DT[out.dtype], int(bool(causal)), float(sm_scale), _stream(q))
-    _check("sage2_attn_fwd", st)
+    st = lib().sage2_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, _DT[q.dtype],
+                                 _DT[out.dtype], int(bool(causal)), float(sm_scale),
+                                 _QKF[qk_bits], int(bool(smooth_v)), _stream(q))
+    _check("sage2_attn_fwd_ex", st)
     return out
 
 
@@ -226,10 +260,14 @@ def sage2_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ca
 
 
 def sage2_debug_qk_s32(q_i4: torch.Tensor, k_i4: torch.Tensor, N: int) -> torch.Tensor:
-    """Raw int32 tiles of q_i4 . k_i4^T (e4m3 codes of INT4 values) through the
-    tcgen05 FP8 path of the attention kernel."""
+    """Raw int32 tiles of q_i4 . k_i4^T through the attention kernel's tensor
+    path: the FP8 path for uint8 e4m3 codes of INT4 values, the 8-bit integer
+    path for int8 values (the INT8 variant)."""
     B, H, Np, d = q_i4.shape
+    if k_i4.dtype != q_i4.dtype:
+        raise ValueError("q_i4 and k_i4 must have the same payload format")
     s = torch.empty(B, H, Np, Np, dtype=torch.int32, device=q_i4.device)
-    st = lib().sage2_debug_qk_s32(_ptr(q_i4), _ptr(k_i4), B, H, N, d, _ptr(s), _stream(q_i4))
-    _check("sage2_debug_qk_s32", st)
+    st = lib().sage2_debug_qk_s32_ex(_ptr(q_i4), _ptr(k_i4), B, H, N, d,
+                                     _QKF[_qk_bits_of(q_i4)], _ptr(s), _stream(q_i4))
+    _check("sage2_debug_qk_s32_ex", st)
     return s

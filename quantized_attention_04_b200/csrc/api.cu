@@ -107,6 +107,9 @@ static sage2_status check_ptrs(P... ps) {
   return SAGE2_OK;
 }
 
+static bool valid_qk_format(int f) { return f == SAGE2_QK_INT4 || f == SAGE2_QK_INT8; }
+static int qk_bits_of(int f) { return f == SAGE2_QK_INT8 ? 8 : 4; }
+
 static sage2_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return SAGE2_OK;
   if (e == cudaErrorMemoryAllocation) return SAGE2_ERR_NO_MEM;
@@ -116,7 +119,7 @@ static sage2_status from_cuda(cudaError_t e) {
 // ------------------------------------------------------------ workspace
 struct Workspace {
   size_t off_q_i4, off_k_i4, off_vt, off_qs, off_ks, off_qm, off_km, off_corr, off_vs, off_part,
-      off_amax, off_qsplit, total;
+      off_amax, off_qsplit, off_vmean, total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -142,6 +145,7 @@ static Workspace layout(const Dims& g) {
   w.off_part = take(BH * NB * d * 4);
   w.off_amax = take(BH * d * 4);
   w.off_qsplit = take(3 * BH * ((NB + 127) / 128) * 128 * d * 2);
+  w.off_vmean = take(BH * d * 4);
   w.total = o;
   return w;
 }
@@ -172,14 +176,15 @@ using namespace sage2;
 
 extern "C" {
 
-sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int B, int H, int N,
-                                   int d, uint8_t* q_i4, float* q_scale, float* q_mean,
-                                   uint8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
-                                   sage2_stream_t stream) {
+sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, int B, int H, int N,
+                                      int d, uint8_t* q_i4, float* q_scale, float* q_mean,
+                                      uint8_t* k_i4, float* k_scale, float* k_mean,
+                                      float* qk_corr, int qk_format, sage2_stream_t stream) {
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;
   if (dtype != SAGE2_F16 && dtype != SAGE2_BF16) return SAGE2_ERR_INVALID_ARG;
+  if (!valid_qk_format(qk_format)) return SAGE2_ERR_INVALID_ARG;
   s = check_ptrs(q, k, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
   if (s != SAGE2_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -196,36 +201,64 @@ sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int 
                                           part_bytes + split_bytes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
   QKArgs a{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean,
-           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, 0};
+           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, 0,
+           qk_bits_of(qk_format)};
   e = launch_smooth_quant_qk(a, st);
   const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
 }
 
-sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d, uint8_t* v_fp8_t,
-                           float* v_scale, sage2_stream_t stream) {
+sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int B, int H, int N,
+                                   int d, uint8_t* q_i4, float* q_scale, float* q_mean,
+                                   uint8_t* k_i4, float* k_scale, float* k_mean, float* qk_corr,
+                                   sage2_stream_t stream) {
+  return sage2_smooth_quant_qk_ex(q, k, dtype, B, H, N, d, q_i4, q_scale, q_mean, k_i4, k_scale,
+                                  k_mean, qk_corr, SAGE2_QK_INT4, stream);
+}
+
+sage2_status sage2_quant_v_ex(const void* v, int dtype, int B, int H, int N, int d,
+                              uint8_t* v_fp8_t, float* v_scale, float* v_mean,
+                              sage2_stream_t stream) {
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;
   if (dtype != SAGE2_F16 && dtype != SAGE2_BF16) return SAGE2_ERR_INVALID_ARG;
   s = check_ptrs(v, v_fp8_t, v_scale);
   if (s != SAGE2_OK) return s;
+  if (v_mean && !aligned16(v_mean)) return SAGE2_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint32_t* amax = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&amax), g.BH * d * 4, st);
+  // scratch: the per-channel |V| maximum and, with smoothing, the mean partial sums
+  const size_t amax_bytes = up256(static_cast<size_t>(g.BH) * d * 4);
+  const size_t part_bytes = v_mean ? up256(static_cast<size_t>(g.BH) * g.NB * d * 4) : 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE2_ERR_CUDA;
+  cudaMemPool_t pool = device_pool(dev);
+  if (!pool) return SAGE2_ERR_CUDA;
+  uint8_t* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch),
+                                          amax_bytes + part_bytes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
-  VArgs a{v, dtype, B, H, N, d, g.Np, g.NB, v_fp8_t, v_scale, amax};
+  VArgs a{v, dtype, B, H, N, d, g.Np, g.NB, v_fp8_t, v_scale,
+          reinterpret_cast<uint32_t*>(scratch), v_mean,
+          v_mean ? reinterpret_cast<float*>(scratch + amax_bytes) : nullptr};
   e = launch_quant_v(a, st);
-  const cudaError_t e2 = cudaFreeAsync(amax, st);
+  const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
 }
 
-sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
-                                      const uint8_t* k_i4, const float* k_scale,
-                                      const float* qk_corr, const uint8_t* v_fp8_t,
-                                      const float* v_scale, void* o, int o_dtype, int B, int H,
-                                      int N, int d, int causal, float sm_scale,
-                                      sage2_stream_t stream) {
+sage2_status sage2_quant_v(const void* v, int dtype, int B, int H, int N, int d, uint8_t* v_fp8_t,
+                           float* v_scale, sage2_stream_t stream) {
+  return sage2_quant_v_ex(v, dtype, B, H, N, d, v_fp8_t, v_scale, nullptr, stream);
+}
+
+sage2_status sage2_attn_fwd_quantized_ex(const uint8_t* q_i4, const float* q_scale,
+                                         const uint8_t* k_i4, const float* k_scale,
+                                         const float* qk_corr, const uint8_t* v_fp8_t,
+                                         const float* v_scale, const float* v_mean, void* o,
+                                         int o_dtype, int B, int H, int N, int d, int causal,
+                                         float sm_scale, int qk_format, sage2_stream_t stream) {
+  if (!valid_qk_format(qk_format)) return SAGE2_ERR_INVALID_ARG;
+  if (v_mean && !aligned16(v_mean)) return SAGE2_ERR_MISALIGNED;
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;
@@ -235,8 +268,20 @@ sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
   s = check_ptrs(q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale, o);
   if (s != SAGE2_OK) return s;
   AttnArgs a{q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale, o, o_dtype,
-             B,    H,       N,    d,       g.Np,    g.NB,    causal,  sm_scale};
+             B,    H,       N,    d,       g.Np,    g.NB,    causal,  sm_scale,
+             qk_bits_of(qk_format), v_mean};
   return from_cuda(launch_attn(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
+                                      const uint8_t* k_i4, const float* k_scale,
+                                      const float* qk_corr, const uint8_t* v_fp8_t,
+                                      const float* v_scale, void* o, int o_dtype, int B, int H,
+                                      int N, int d, int causal, float sm_scale,
+                                      sage2_stream_t stream) {
+  return sage2_attn_fwd_quantized_ex(q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale,
+                                     nullptr, o, o_dtype, B, H, N, d, causal, sm_scale,
+                                     SAGE2_QK_INT4, stream);
 }
 
 size_t sage2_workspace_bytes(int B, int H, int N, int d) {
@@ -245,9 +290,12 @@ size_t sage2_workspace_bytes(int B, int H, int N, int d) {
   return layout(g).total;
 }
 
-sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
-                            int N, int d, int dtype, int o_dtype, int causal, float sm_scale,
-                            sage2_stream_t stream) {
+sage2_status sage2_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, int B,
+                               int H, int N, int d, int dtype, int o_dtype, int causal,
+                               float sm_scale, int qk_format, int smooth_v,
+                               sage2_stream_t stream) {
+  if (!valid_qk_format(qk_format)) return SAGE2_ERR_INVALID_ARG;
+  if (smooth_v != 0 && smooth_v != 1) return SAGE2_ERR_INVALID_ARG;
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;
@@ -279,12 +327,15 @@ sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o
   float* vs = reinterpret_cast<float*>(ws + w.off_vs);
   float* part = reinterpret_cast<float*>(ws + w.off_part);
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
+  float* vmean = smooth_v ? reinterpret_cast<float*>(ws + w.off_vmean) : nullptr;
+  const int qk_bits = qk_bits_of(qk_format);
 
   QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
-            ws + w.off_qsplit, causal};
-  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax};
+            ws + w.off_qsplit, causal, qk_bits};
+  // the V mean reuses the K-mean scratch: stream order puts it after the K mean
+  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, vmean, part};
   AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
-              sm_scale};
+              sm_scale, qk_bits, vmean};
   e = launch_smooth_quant_qk(qa, st);
   if (e == cudaSuccess) e = launch_quant_v(va, st);
   if (e == cudaSuccess) e = launch_attn(aa, st);
@@ -292,8 +343,16 @@ sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o
   return from_cuda(e != cudaSuccess ? e : e2);
 }
 
-sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
-                                int d, int32_t* s_out, sage2_stream_t stream) {
+sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int N, int d, int dtype, int o_dtype, int causal, float sm_scale,
+                            sage2_stream_t stream) {
+  return sage2_attn_fwd_ex(q, k, v, o, B, H, N, d, dtype, o_dtype, causal, sm_scale,
+                           SAGE2_QK_INT4, 0, stream);
+}
+
+sage2_status sage2_debug_qk_s32_ex(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
+                                   int d, int qk_format, int32_t* s_out, sage2_stream_t stream) {
+  if (!valid_qk_format(qk_format)) return SAGE2_ERR_INVALID_ARG;
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;
@@ -301,8 +360,13 @@ sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B,
   if (g.BH > 65535) return SAGE2_ERR_UNSUPPORTED;
   s = check_ptrs(q_i4, k_i4, s_out);
   if (s != SAGE2_OK) return s;
-  return from_cuda(launch_debug_qk(q_i4, k_i4, B, H, g.Np, d, s_out,
+  return from_cuda(launch_debug_qk(q_i4, k_i4, B, H, g.Np, d, qk_bits_of(qk_format), s_out,
                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
+                                int d, int32_t* s_out, sage2_stream_t stream) {
+  return sage2_debug_qk_s32_ex(q_i4, k_i4, B, H, N, d, SAGE2_QK_INT4, s_out, stream);
 }
 
 sage2_status sage2_check_device_error(sage2_stream_t stream) {

@@ -42,6 +42,8 @@ constexpr int kStages = 4;
 constexpr int kThreads = 512;
 constexpr int kSegStride = 36;                   // floats between the 32-key groups in shared memory
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+constexpr uint32_t kMagicBits = 0x4B400000u;     // 1.5 * 2^23 (INT8 variant, see dequant16)
+constexpr float kMagic = 12582912.0f;
 
 template <int D>
 struct __align__(1024) AttnSmem {
@@ -56,6 +58,7 @@ struct __align__(1024) AttnSmem {
   float ksc[kStages][4 * kSegStride];
   float qsc[128];                  // q_scale of the block's rows
   float vsc[D];                     // v_scale (correction warpgroup)
+  float vmean[D];                   // token mean of V when V was smoothed, else 0
   float alpha[4][128];              // per-row rescale factor of tile t in slot t%4 (softmax -> correction)
   float lsum[128];                  // final row sums (448-scaled), softmax -> correction
   uint64_t q_full;
@@ -103,11 +106,22 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
 // warpgroup for the first, kBarExpB + q the other way round.
 constexpr int kBarExpA = 3, kBarExpB = 7;
 
+// The score S_ij as a float.  INT4 (QB = 4): S comes out of the FP8 tensor
+// path as an fp32 integer: the INT4 values are exact in e4m3, every product
+// (|.| <= 49) and partial sum (|.| <= 49*128 < 2^13) is an integer the fp32
+// accumulator holds exactly.  INT8 (QB = 8): S is s32 (|S| <= 127^2*128 <
+// 2^22); its bits plus 0x4B400000, read as a float, are exactly 1.5*2^23 + S,
+// and subtracting 1.5*2^23 is exact.
+template <int QB>
+__device__ __forceinline__ float2 s_pair(uint32_t a, uint32_t b) {
+  if (QB == 4) return make_float2(__uint_as_float(a), __uint_as_float(b));
+  return __fadd2_rn(make_float2(__uint_as_float(a + kMagicBits), __uint_as_float(b + kMagicBits)),
+                    make_float2(-kMagic, -kMagic));
+}
+
 // Dequantise + correct the 16 keys 4m..4m+3 (m = 0..3) of both rows held in
-// one .16x256b.x8 load: x' = sq_i * (sk_j * S_ij) + C_j.  S comes out of the
-// FP8 tensor path as an fp32 integer: the INT4 values are exact in e4m3, every
-// product (|.| <= 49) and partial sum (|.| <= 49*128 < 2^13) is an integer the
-// fp32 accumulator holds exactly.
+// one .16x256b.x8 load: x' = sq_i * (sk_j * S_ij) + C_j.
+template <int QB>
 __device__ __forceinline__ void dequant16(const uint32_t (&sr)[32], const float* ck,
                                           const float* kk, float2 a0, float2 a1, float* x0,
                                           float* x1) {
@@ -118,10 +132,10 @@ __device__ __forceinline__ void dequant16(const uint32_t (&sr)[32], const float*
     const float2 kxy = make_float2(k4.x, k4.y), kzw = make_float2(k4.z, k4.w);
     const float2 cxy = make_float2(c4.x, c4.y), czw = make_float2(c4.z, c4.w);
     const uint32_t* q = sr + 8 * m;
-    const float2 r00 = __ffma2_rn(a0, __fmul2_rn(kxy, make_float2(__uint_as_float(q[0]), __uint_as_float(q[1]))), cxy);
-    const float2 r01 = __ffma2_rn(a0, __fmul2_rn(kzw, make_float2(__uint_as_float(q[4]), __uint_as_float(q[5]))), czw);
-    const float2 r10 = __ffma2_rn(a1, __fmul2_rn(kxy, make_float2(__uint_as_float(q[2]), __uint_as_float(q[3]))), cxy);
-    const float2 r11 = __ffma2_rn(a1, __fmul2_rn(kzw, make_float2(__uint_as_float(q[6]), __uint_as_float(q[7]))), czw);
+    const float2 r00 = __ffma2_rn(a0, __fmul2_rn(kxy, s_pair<QB>(q[0], q[1])), cxy);
+    const float2 r01 = __ffma2_rn(a0, __fmul2_rn(kzw, s_pair<QB>(q[4], q[5])), czw);
+    const float2 r10 = __ffma2_rn(a1, __fmul2_rn(kxy, s_pair<QB>(q[2], q[3])), cxy);
+    const float2 r11 = __ffma2_rn(a1, __fmul2_rn(kzw, s_pair<QB>(q[6], q[7])), czw);
     x0[4 * m] = r00.x;
     x0[4 * m + 1] = r00.y;
     x0[4 * m + 2] = r01.x;
@@ -210,13 +224,13 @@ __device__ __forceinline__ void store8(void* out, size_t idx, const float (&f)[8
   }
 }
 
-template <int D, int OT>
+template <int D, int OT, int QB>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                const float* __restrict__ k_scale, const float* __restrict__ qk_corr,
-               const float* __restrict__ v_scale, void* __restrict__ out, int N, int Np, int NB,
-               int causal, float L) {
+               const float* __restrict__ v_scale, const float* __restrict__ v_mean,
+               void* __restrict__ out, int N, int Np, int NB, int causal, float L) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -293,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128);   // INT4 values in e4m3
+      // INT4 values as e4m3 codes on the FP8 path; INT8 values on the 8-bit integer path
+      constexpr uint32_t idesc_qk = QB == 4 ? idesc_e4m3_f32(128, 128) : idesc_i8_s32(128, 128);
       constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, D);
       // descriptors are built once; a k-step or a stage only moves the start
       // address field (16-byte units; shared memory is < 256 KB, no carry)
@@ -312,7 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t kb = dk + s * kStageK;
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk) mma_f8_ss(tmem + b * 128, dq + 2 * kk, kb + 2 * kk, idesc_qk, kk > 0);
+        for (int kk = 0; kk < D / 32; ++kk) {
+          if (QB == 4) mma_f8_ss(tmem + b * 128, dq + 2 * kk, kb + 2 * kk, idesc_qk, kk > 0);
+          else mma_i8_ss(tmem + b * 128, dq + 2 * kk, kb + 2 * kk, idesc_qk, kk > 0);
+        }
         tc_commit(&sm.s_full[b]);
         return true;
       };
@@ -399,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // also carries the MMA thread's release after it acquired kv_full
         const float* ck = sm.corr[s] + kSegStride * g;
         const float* kk = sm.ksc[s] + kSegStride * g;
-        dequant16(sA, ck, kk, a02, a12, x0, x1);
-        dequant16(sB, ck + 16, kk + 16, a02, a12, x0 + 16, x1 + 16);
+        dequant16<QB>(sA, ck, kk, a02, a12, x0, x1);
+        dequant16<QB>(sB, ck + 16, kk + 16, a02, a12, x0 + 16, x1 + 16);
       }
       if ((causal && t == qt) || (tail && t == NB - 1)) {
 #pragma unroll
@@ -464,7 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (warp & 3) * 32 + lane;
     const int row = qt * 128 + r;
     const uint32_t tI = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + 256;
-    for (int i = r; i < D; i += 128) sm.vsc[i] = v_scale[static_cast<size_t>(bh) * D + i];
+    for (int i = r; i < D; i += 128) {
+      sm.vsc[i] = v_scale[static_cast<size_t>(bh) * D + i];
+      sm.vmean[i] = v_mean ? v_mean[static_cast<size_t>(bh) * D + i] : 0.f;
+    }
     named_bar_sync(1, 128);
     float acc[D];
 #pragma unroll
@@ -496,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D; c += 8) {
         float f[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) f[u] = acc[c + u] * sm.vsc[c + u] * inv;
+        for (int u = 0; u < 8; ++u) f[u] = acc[c + u] * sm.vsc[c + u] * inv + sm.vmean[c + u];
         store8<OT>(out, obase + c, f);
       }
     }
@@ -509,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int OT>
+template <int D, int OT, int QB>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   alignas(64) CUtensorMap tq, tk, tv;
   const int BH = a.B * a.H;
@@ -521,24 +542,30 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   e = make_tmap_u8_2d(&tv, a.v_fp8_t, static_cast<uint64_t>(BH) * D, a.Np, D, 128);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(AttnSmem<D>) + 1024;
-  e = cudaFuncSetAttribute(k_attn_fwd<D, OT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(k_attn_fwd<D, OT, QB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const float L = a.sm_scale * 1.4426950408889634f;
-  k_attn_fwd<D, OT><<<dim3(a.NB, BH), kThreads, smem, st>>>(
-      tq, tk, tv, a.q_scale, a.k_scale, a.qk_corr, a.v_scale, a.o, a.N, a.Np, a.NB, a.causal, L);
+  k_attn_fwd<D, OT, QB><<<dim3(a.NB, BH), kThreads, smem, st>>>(
+      tq, tk, tv, a.q_scale, a.k_scale, a.qk_corr, a.v_scale, a.v_mean, a.o, a.N, a.Np, a.NB,
+      a.causal, L);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+template <int QB>
+static cudaError_t launch_attn_q(const AttnArgs& a, cudaStream_t st) {
   if (a.d == 64) {
-    if (a.o_dtype == 0) return launch_attn_t<64, 0>(a, st);
-    if (a.o_dtype == 1) return launch_attn_t<64, 1>(a, st);
-    return launch_attn_t<64, 2>(a, st);
+    if (a.o_dtype == 0) return launch_attn_t<64, 0, QB>(a, st);
+    if (a.o_dtype == 1) return launch_attn_t<64, 1, QB>(a, st);
+    return launch_attn_t<64, 2, QB>(a, st);
   }
-  if (a.o_dtype == 0) return launch_attn_t<128, 0>(a, st);
-  if (a.o_dtype == 1) return launch_attn_t<128, 1>(a, st);
-  return launch_attn_t<128, 2>(a, st);
+  if (a.o_dtype == 0) return launch_attn_t<128, 0, QB>(a, st);
+  if (a.o_dtype == 1) return launch_attn_t<128, 1, QB>(a, st);
+  return launch_attn_t<128, 2, QB>(a, st);
+}
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+  return a.qk_bits == 8 ? launch_attn_q<8>(a, st) : launch_attn_q<4>(a, st);
 }
 
 }  // namespace sage2

@@ -1,6 +1,7 @@
-// Test kernel: raw tiles of the INT4 product Q^ K^T through the same TMA +
-// tcgen05 FP8 path as the attention kernel (INT4 values in e4m3 codes, fp32
-// accumulator; one 128x128 tile per CTA), written as int32.
+// Test kernel: raw tiles of the integer product Q^ K^T through the same TMA +
+// tcgen05 path as the attention kernel (one 128x128 tile per CTA), written as
+// int32: INT4 values as e4m3 codes on the FP8 path (exact fp32 integer sums,
+// converted), or INT8 values on the 8-bit integer path (s32 accumulator).
 // Lets the integer matrix product ("4-bit matrix multiplication", SageAttention2
 // abstract page, Abstract) be checked bit for bit on its own.
 #include <cuda.h>
@@ -10,7 +11,7 @@
 
 namespace sage2 {
 
-template <int D>
+template <int D, int QB>
 __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CUtensorMap tm_q,
                                                       const __grid_constant__ CUtensorMap tm_k,
                                                       int Np, int32_t* __restrict__ s_out) {
@@ -46,11 +47,16 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
     tma_load_2d(sk, &tm_k, &bar_load, 0, bh * Np + kt * 128);
     if (mbar_wait(&bar_load, 0, &abort_flag)) {
       tc_fence_after();
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, 128);
+      constexpr uint32_t idesc = QB == 4 ? idesc_e4m3_f32(128, 128) : idesc_i8_s32(128, 128);
 #pragma unroll
-      for (int kk = 0; kk < D / 32; ++kk)
-        mma_f8_ss(tmem, smem_desc_kmajor(sq + 32 * kk, D), smem_desc_kmajor(sk + 32 * kk, D),
-                  idesc, kk > 0);
+      for (int kk = 0; kk < D / 32; ++kk) {
+        if (QB == 4)
+          mma_f8_ss(tmem, smem_desc_kmajor(sq + 32 * kk, D), smem_desc_kmajor(sk + 32 * kk, D),
+                    idesc, kk > 0);
+        else
+          mma_i8_ss(tmem, smem_desc_kmajor(sq + 32 * kk, D), smem_desc_kmajor(sk + 32 * kk, D),
+                    idesc, kk > 0);
+      }
       tc_commit(&bar_mma);
     }
   }
@@ -68,8 +74,9 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
 #pragma unroll
       for (int u = 0; u < 32; u += 4)
         *reinterpret_cast<int4*>(dst + c0 + u) =
-            make_int4(__float2int_rn(__uint_as_float(v[u])), __float2int_rn(__uint_as_float(v[u + 1])),
-                      __float2int_rn(__uint_as_float(v[u + 2])), __float2int_rn(__uint_as_float(v[u + 3])));
+            QB == 4 ? make_int4(__float2int_rn(__uint_as_float(v[u])), __float2int_rn(__uint_as_float(v[u + 1])),
+                                __float2int_rn(__uint_as_float(v[u + 2])), __float2int_rn(__uint_as_float(v[u + 3])))
+                    : make_int4(v[u], v[u + 1], v[u + 2], v[u + 3]);
     }
   }
   tc_fence_before();
@@ -80,7 +87,7 @@ __global__ void __launch_bounds__(128) k_debug_qk_s32(const __grid_constant__ CU
   }
 }
 
-template <int D>
+template <int D, int QB>
 static cudaError_t launch_debug_t(const uint8_t* q_i4, const uint8_t* k_i4, int BH, int Np,
                                   int32_t* s_out, cudaStream_t st) {
   alignas(64) CUtensorMap tq, tk;
@@ -90,14 +97,17 @@ static cudaError_t launch_debug_t(const uint8_t* q_i4, const uint8_t* k_i4, int 
   if (e != cudaSuccess) return e;
   const int smem = 2 * 128 * D + 1024;
   const int nt = Np / 128;
-  k_debug_qk_s32<D><<<dim3(nt, nt, BH), 128, smem, st>>>(tq, tk, Np, s_out);
+  k_debug_qk_s32<D, QB><<<dim3(nt, nt, BH), 128, smem, st>>>(tq, tk, Np, s_out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int Np, int d,
-                            int32_t* s_out, cudaStream_t st) {
-  return d == 64 ? launch_debug_t<64>(q_i4, k_i4, B * H, Np, s_out, st)
-                 : launch_debug_t<128>(q_i4, k_i4, B * H, Np, s_out, st);
+                            int qk_bits, int32_t* s_out, cudaStream_t st) {
+  if (qk_bits == 8)
+    return d == 64 ? launch_debug_t<64, 8>(q_i4, k_i4, B * H, Np, s_out, st)
+                   : launch_debug_t<128, 8>(q_i4, k_i4, B * H, Np, s_out, st);
+  return d == 64 ? launch_debug_t<64, 4>(q_i4, k_i4, B * H, Np, s_out, st)
+                 : launch_debug_t<128, 4>(q_i4, k_i4, B * H, Np, s_out, st);
 }
 
 }  // namespace sage2

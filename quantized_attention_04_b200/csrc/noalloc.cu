@@ -99,10 +99,10 @@ extern "C" sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, con
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
 
   QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
-            ws + w.off_qsplit, causal};
-  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax};  // amax is cleared on the stream
+            ws + w.off_qsplit, causal, 4};
+  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, nullptr, nullptr};  // amax is cleared on the stream
   AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
-              sm_scale};
+              sm_scale, 4, nullptr};
   e = launch_smooth_quant_qk(qa, st);
   if (e == cudaSuccess) e = launch_quant_v(va, st);
   if (e == cudaSuccess) e = launch_attn(aa, st);

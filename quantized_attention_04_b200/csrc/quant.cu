@@ -10,7 +10,10 @@
 // Method: "SageAttention2: Efficient Attention with Thorough Outlier Smoothing
 // and Per-thread INT4 Quantization" (arxiv.science abstract page, Abstract):
 // INT4 (Q,K), FP8 V, smoothing of Q; K smoothing from the title's "outlier
-// smoothing".  Every rounding below is spelled with an explicit IEEE intrinsic
+// smoothing".  Variants: INT8 (Q,K) on [-127, 127] (the predecessor,
+// "SageAttention: Accurate 8-Bit Attention", ainnect summary) and V smoothing
+// (token mean of V subtracted before FP8, "smooth V" in the SageAttention2
+// summary, ainnect.com/research/55).  Every rounding below is spelled with an explicit IEEE intrinsic
 // (__fadd_rn, __fmul_rn, ...) so that no contraction or reassociation changes
 // the payload bits: the summation orders are part of the specification.
 #include <cuda_bf16.h>
@@ -104,7 +107,7 @@ __global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int
 // ---------------------------------------------------------------------------
 // Smoothing + INT4.  grid (NB, B*H, 2): z = 0 quantizes the Q block (after
 // computing its mean), z = 1 the K block (after subtracting kbar).  256 threads.
-template <typename T, int D>
+template <typename T, int D, bool Q8>
 __global__ void __launch_bounds__(256) k_smooth_quant(
     const T* __restrict__ q, const T* __restrict__ k, int N, int Np, int NB,
     const float* __restrict__ kmean, uint8_t* __restrict__ q_i4, float* __restrict__ q_scale,
@@ -158,22 +161,27 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    // Each INT4 value is stored as its e4m3 code: every integer in [-7, 7] is
-    // exact in e4m3, so the FP8 tensor path multiplies the INT4 values exactly
-    // (at the same rate as the 8-bit integer path) and yields S as an fp32
-    // integer.  Zero is stored as +0 (code 0x00).
+    // INT4 (the method): each value in [-7, 7] is stored as its e4m3 code:
+    // every such integer is exact in e4m3, so the FP8 tensor path multiplies
+    // the INT4 values exactly (at the same rate as the 8-bit integer path) and
+    // yields S as an fp32 integer.  Zero is stored as +0 (code 0x00).
+    // INT8 (the variant): values in [-127, 127] as two's-complement bytes.
+    constexpr float kQmax = Q8 ? 127.f : 7.f;
     uint32_t packed = 0;
     float sc = 0.f;
     if (amax > 0.f) {
-      sc = __fdiv_rn(amax, 7.f);
-      const float inv = __fdiv_rn(7.f, amax);
+      sc = __fdiv_rn(amax, kQmax);
+      const float inv = __fdiv_rn(kQmax, amax);
 #pragma unroll
       for (int i = 0; i < CPL; ++i) {
         float v = rintf(__fmul_rn(x[i], inv));
-        v = fminf(fmaxf(v, -7.f), 7.f);
-        const float vi = static_cast<float>(static_cast<int>(v));   // -0 -> +0
-        packed |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(vi, __NV_SATFINITE, __NV_E4M3))
-                  << (8 * i);
+        v = fminf(fmaxf(v, -kQmax), kQmax);
+        const int vi = static_cast<int>(v);                          // -0 -> 0
+        const uint32_t byte =
+            Q8 ? (static_cast<uint32_t>(vi) & 0xFFu)
+               : static_cast<uint32_t>(__nv_cvt_float_to_fp8(static_cast<float>(vi),
+                                                              __NV_SATFINITE, __NV_E4M3));
+        packed |= byte << (8 * i);
       }
     }
     const int srow = is_q ? r : 8 * ((r >> 1) & 15) + 2 * (r >> 5) + (r & 1);
@@ -192,6 +200,7 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
 // like unsigned integers, so atomicMax on the bits is exact.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
+                                                const float* __restrict__ vmean,
                                                 uint32_t* __restrict__ amax_bits) {
   constexpr int TPR = D / 8;
   constexpr int RPB = 256 / TPR;  // rows handled at once by the block
@@ -200,15 +209,18 @@ __global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
   const int r = threadIdx.x / TPR, q8 = threadIdx.x % TPR;
   const int t0 = chunk * 128;
   const int nt = min(128, N - t0);
-  float m[8];
+  float m[8], mu[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = 0.f;
+  for (int i = 0; i < 8; ++i) {
+    m[i] = 0.f;
+    mu[i] = vmean ? vmean[(size_t)bh * D + q8 * 8 + i] : 0.f;   // V smoothing: |V - vbar|
+  }
   const uint4* src = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + t0) * D) + q8;
   for (int t = r; t < nt; t += RPB) {
     float x[8];
     unpack8<T>(__ldg(src + (size_t)t * TPR), x);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(x[i]));
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(__fsub_rn(x[i], mu[i])));
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) red[r][q8 * 8 + i] = m[i];
@@ -225,11 +237,12 @@ __global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
 // consecutive channels, so its shared-memory reads are conflict-free.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N, int Np,
+                                                 const float* __restrict__ vmean,
                                                  const uint32_t* __restrict__ amax_bits,
                                                  uint8_t* __restrict__ vt,
                                                  float* __restrict__ v_scale) {
   __shared__ __align__(16) T tile[128][D];
-  __shared__ float inv[D];
+  __shared__ float inv[D], mu[D];
   const int kt = blockIdx.x, bh = blockIdx.y;
   const int t0 = kt * 128;
   const int nvalid = max(0, min(128, N - t0));
@@ -240,6 +253,7 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
   if (threadIdx.x < D) {
     const float a = __uint_as_float(amax_bits[(size_t)bh * D + threadIdx.x]);
     inv[threadIdx.x] = a > 0.f ? __fdiv_rn(448.f, a) : 0.f;
+    mu[threadIdx.x] = vmean ? vmean[(size_t)bh * D + threadIdx.x] : 0.f;
     if (kt == 0) v_scale[(size_t)bh * D + threadIdx.x] = a > 0.f ? __fdiv_rn(a, 448.f) : 0.f;
   }
   __syncthreads();
@@ -248,7 +262,7 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
   for (int item = warp; item < (D / 32) * 8; item += 8) {
     const int c = (item / 8) * 32 + lane;
     const int tg = item % 8;
-    const float sc = inv[c];
+    const float sc = inv[c], m0 = mu[c];
     uint32_t w[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
@@ -256,8 +270,8 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int r = tg * 16 + p * 4 + h * 2;
-        const float x0 = (r < nvalid) ? __fmul_rn(to_f32(tile[r][c]), sc) : 0.f;
-        const float x1 = (r + 1 < nvalid) ? __fmul_rn(to_f32(tile[r + 1][c]), sc) : 0.f;
+        const float x0 = (r < nvalid) ? __fmul_rn(__fsub_rn(to_f32(tile[r][c]), m0), sc) : 0.f;
+        const float x1 = (r + 1 < nvalid) ? __fmul_rn(__fsub_rn(to_f32(tile[r + 1][c]), m0), sc) : 0.f;
         const __nv_fp8x2_storage_t two =
             __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
         word |= static_cast<uint32_t>(two) << (16 * h);
@@ -282,9 +296,14 @@ static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
   k_mean_partial<T, D><<<dim3((nchunks + WPB - 1) / WPB, BH), 256, 0, st>>>(
       static_cast<const T*>(a.k), a.N, nchunks, a.mean_part);
   k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, nchunks, a.N, D, a.k_mean);
-  k_smooth_quant<T, D><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
-      static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
-      a.q_scale, a.q_mean, a.k_i4, a.k_scale);
+  if (a.qk_bits == 8)
+    k_smooth_quant<T, D, true><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
+        a.q_scale, a.q_mean, a.k_i4, a.k_scale);
+  else
+    k_smooth_quant<T, D, false><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
+        a.q_scale, a.q_mean, a.k_i4, a.k_scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_qk_corr_t<T, D>(a, st);
@@ -300,9 +319,17 @@ static cudaError_t launch_v_t(const VArgs& a, cudaStream_t st) {
   const int BH = a.B * a.H;
   cudaError_t e = cudaMemsetAsync(a.amax_bits, 0, sizeof(uint32_t) * BH * D, st);
   if (e != cudaSuccess) return e;
-  k_v_amax<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.amax_bits);
+  if (a.v_mean) {
+    // V smoothing: the per-channel token mean, with the fixed order of the K mean
+    constexpr int WPB = 256 / (D / 8);
+    k_mean_partial<T, D><<<dim3((a.NB + WPB - 1) / WPB, BH), 256, 0, st>>>(
+        static_cast<const T*>(a.v), a.N, a.NB, a.mean_part);
+    k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, a.NB, a.N, D, a.v_mean);
+  }
+  k_v_amax<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.v_mean,
+                                                 a.amax_bits);
   k_v_quant<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.Np,
-                                                  a.amax_bits, a.v_fp8_t, a.v_scale);
+                                                  a.v_mean, a.amax_bits, a.v_fp8_t, a.v_scale);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,7 @@ struct QKArgs {
   float* mean_part;        // scratch [B*H, NB, d]
   void* qbar_split;        // scratch [3][B*H][NBc*128][d] in the input dtype (NBc = ceil(NB/128))
   int skip_masked_corr;    // 1: skip correction blocks a causal mask hides
+  int qk_bits;             // 4: INT4 values as e4m3 codes; 8: INT8 values (two's complement)
 };
 
 struct VArgs {
@@ -32,6 +33,8 @@ struct VArgs {
   uint8_t* v_fp8_t;
   float* v_scale;
   uint32_t* amax_bits;     // scratch [B*H, d]
+  float* v_mean;           // nullptr: no V smoothing; else the per-channel token mean [B*H, d]
+  float* mean_part;        // scratch [B*H, NB, d] for the V mean (when v_mean is set)
 };
 
 struct AttnArgs {
@@ -47,13 +50,15 @@ struct AttnArgs {
   int B, H, N, d, Np, NB;
   int causal;
   float sm_scale;
+  int qk_bits;             // 4 or 8 (payload format, see QKArgs)
+  const float* v_mean;     // nullptr: V was not smoothed
 };
 
 cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int Np, int d,
-                            int32_t* s_out, cudaStream_t st);
+                            int qk_bits, int32_t* s_out, cudaStream_t st);
 
 // General tiled tensor map: `rank` dims (innermost first, in elements), the
 // byte strides of dims 1..rank-1, the box (elements), element size 1/2/4 B and

@@ -27,10 +27,11 @@ def np32(t: torch.Tensor) -> np.ndarray:
     return t.detach().to(torch.float32).cpu().numpy()
 
 
-def oracle_head(q, k, v, b, h, causal, sm_scale, q_blocks=None):
+def oracle_head(q, k, v, b, h, causal, sm_scale, q_blocks=None, qk_bits=4, smooth_v=False):
     """Oracle payloads and output rows of head (b, h); q/k/v are [B,H,N,d]."""
     Q, K, V = np32(q[b, h]), np32(k[b, h]), np32(v[b, h])
-    pay, O, amb, rows = orc.sage2_head(Q, K, V, causal, sm_scale, q_blocks=q_blocks)
+    pay, O, amb, rows = orc.sage2_head(Q, K, V, causal, sm_scale, q_blocks=q_blocks,
+                                       qk_bits=qk_bits, smooth_v=smooth_v)
     return pay, O, amb, rows
 
 

@@ -29,7 +29,10 @@ def test_header_declares_the_boundary():
     names = _declared()
     for must in ("sage2_attn_fwd", "sage2_smooth_quant_qk", "sage2_quant_v",
                  "sage2_attn_fwd_quantized", "sage2_debug_qk_s32", "sage2_workspace_bytes",
-                 "sage2_check_device_error", "sage2_status_string"):
+                 "sage2_check_device_error", "sage2_status_string",
+                 # the variants (INT8 Q/K, V smoothing)
+                 "sage2_attn_fwd_ex", "sage2_smooth_quant_qk_ex", "sage2_quant_v_ex",
+                 "sage2_attn_fwd_quantized_ex", "sage2_debug_qk_s32_ex"):
         assert must in names
 
 
@@ -84,6 +87,30 @@ def test_validation_other_entries(L):
     assert L.sage2_debug_qk_s32(P, P, 1, 1, 10, 64, 0, None) == 1
 
 
+def test_validation_variant_entries(L):
+    def attn_ex(fmt=0, smooth=0, **kw):
+        a = dict(q=P, k=P, v=P, o=P, B=1, H=2, N=256, d=64, dt=0, odt=2, causal=0, sm=0.125)
+        a.update(kw)
+        return L.sage2_attn_fwd_ex(a["q"], a["k"], a["v"], a["o"], a["B"], a["H"], a["N"], a["d"],
+                                   a["dt"], a["odt"], a["causal"], a["sm"], fmt, smooth, None)
+    assert attn_ex(fmt=2) == 1
+    assert attn_ex(fmt=-1) == 1
+    assert attn_ex(smooth=2) == 1
+    assert attn_ex(fmt=1, d=96) == 2
+    assert attn_ex(fmt=1, q=P + 4) == 3
+    z = [P] * 7
+    assert L.sage2_smooth_quant_qk_ex(P, P, 0, 1, 1, 10, 64, *z, 3, None) == 1
+    assert L.sage2_smooth_quant_qk_ex(P, P, 0, 1, 1, 0, 64, *z, 1, None) == 1
+    assert L.sage2_quant_v_ex(P, 0, 1, 1, 10, 64, P, P, P + 8, None) == 3     # misaligned v_mean
+    assert L.sage2_quant_v_ex(P, 0, 1, 1, 10, 64, P, 0, P, None) == 1
+    assert L.sage2_attn_fwd_quantized_ex(P, P, P, P, P, P, P, P, P, 2, 1, 1, 10, 64, 0, 0.1, 5,
+                                         None) == 1
+    assert L.sage2_attn_fwd_quantized_ex(P, P, P, P, P, P, P, P + 4, P, 2, 1, 1, 10, 64, 0, 0.1, 1,
+                                         None) == 3
+    assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 7, P, None) == 1
+    assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 1, 0, None) == 1
+
+
 def test_workspace_bytes(L):
     def expect(B, H, N, d):
         up = lambda x: (x + 255) // 256 * 256
@@ -92,7 +119,7 @@ def test_workspace_bytes(L):
         BH = B * H
         parts = [BH * Np * d, BH * Np * d, BH * d * Np, BH * Np * 4, BH * Np * 4,
                  BH * NB * d * 4, BH * d * 4, BH * NB * Np * 4, BH * d * 4, BH * NB * d * 4,
-                 BH * d * 4, 3 * BH * ((NB + 127) // 128) * 128 * d * 2]
+                 BH * d * 4, 3 * BH * ((NB + 127) // 128) * 128 * d * 2, BH * d * 4]
         return sum(up(p) for p in parts)
     for shape in [(1, 2, 256, 64), (2, 8, 2048, 128), (1, 24, 17776, 64), (1, 1, 1, 128)]:
         assert L.sage2_workspace_bytes(*shape) == expect(*shape)
