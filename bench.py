@@ -173,7 +173,7 @@ def recorded_traffic(workload: str):
 
 
 # ---------------------------------------------------------------- oracle leg
-def oracle_sample(cfg, q, k, v, n_blocks: int):
+def oracle_sample(cfg, q, k, v, n_blocks: int, qk_bits: int = 4, smooth_v: bool = False):
     """Time the CPU oracle on head (0,0): its payloads plus n_blocks query
     blocks spread over the sequence.  Returns (ops, seconds, description)."""
     from oracle import sage2_oracle as orc
@@ -185,7 +185,7 @@ def oracle_sample(cfg, q, k, v, n_blocks: int):
     V = v[0, 0].float().numpy()
     sm = 1.0 / math.sqrt(d)
     t0 = time.perf_counter()
-    orc.sage2_head(Q, K, V, cfg.causal, sm, q_blocks=blocks)
+    orc.sage2_head(Q, K, V, cfg.causal, sm, q_blocks=blocks, qk_bits=qk_bits, smooth_v=smooth_v)
     dt = time.perf_counter() - t0
     ops = 0.0
     for b in blocks:
@@ -208,9 +208,9 @@ def run_reference(args, cfg, world, rank):
     times, opss = [], []
     desc = ""
     for _ in range(args.warmup):
-        oracle_sample(cfg, q, k, v, 1)
+        oracle_sample(cfg, q, k, v, 1, args.qk_bits, args.smooth_v)
     for _ in range(args.steps):
-        ops, dt, desc = oracle_sample(cfg, q, k, v, args.ref_blocks)
+        ops, dt, desc = oracle_sample(cfg, q, k, v, args.ref_blocks, args.qk_bits, args.smooth_v)
         times.append(dt)
         opss.append(ops)
     value = sum(opss) / sum(times) / 1e12
@@ -245,21 +245,23 @@ def run_sage2(args, cfg, world, rank, local):
     od = torch.empty_like(qd)
     stream = torch.cuda.current_stream(dev)
 
+    variant = ("int4" if args.qk_bits == 4 else "int8") + ("+smooth_v" if args.smooth_v else "")
     # Payload buffers are allocated once, by the caller, as the C ABI allows.
-    pay = qa.sage2_smooth_quant_qk(qd, kd)
-    vpay = qa.sage2_quant_v(vd)
+    pay = qa.sage2_smooth_quant_qk(qd, kd, qk_bits=args.qk_bits)
+    vpay = qa.sage2_quant_v(vd, smooth=args.smooth_v)
     # The timed step runs the three stage calls of the C ABI (the same kernels,
     # in the same order, as sage2_attn_fwd) so that the attention launch can be
     # bracketed by its own events on the launching stream.
     attn_ev = []
 
     def step(record: bool):
-        qa.sage2_smooth_quant_qk(qd, kd, out=pay)
-        qa.sage2_quant_v(vd, out=vpay)
+        qa.sage2_smooth_quant_qk(qd, kd, out=pay, qk_bits=args.qk_bits)
+        qa.sage2_quant_v(vd, out=vpay, smooth=args.smooth_v)
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        qa.sage2_attn_fwd_quantized(pay, vpay[0], vpay[1], cfg.N, cfg.causal, sm, out=od)
+        qa.sage2_attn_fwd_quantized(pay, vpay[0], vpay[1], cfg.N, cfg.causal, sm, out=od,
+                                    v_mean=vpay[2] if args.smooth_v else None)
         if record:
             e1.record(stream)
             attn_ev.append((e0, e1))
@@ -296,7 +298,8 @@ def run_sage2(args, cfg, world, rank, local):
     fp8_peak = bf16_peak * 2.0   # dense fp8/int8 : bf16 nominal ratio 4.5 : 2.25
     attn_tflops = cfg.ops() / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": attn_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": attn_tflops / fp8_peak, "traffic": recorded_traffic(cfg.name),
+                "frac": attn_tflops / fp8_peak,
+                "traffic": recorded_traffic(cfg.name) if variant == "int4" else None,
                 "kernel": "k_attn_fwd", "kernel_ms": attn_ms,
                 "peak_source": f"{peak_src} bf16 burst x 2 (fp8/int8 dense : bf16 dense)"}
 
@@ -310,7 +313,8 @@ def run_sage2(args, cfg, world, rank, local):
             qd.copy_(qh, non_blocking=True)
             kd.copy_(kh, non_blocking=True)
             vd.copy_(vh, non_blocking=True)
-            qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out=od)
+            qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out=od,
+                              qk_bits=args.qk_bits, smooth_v=args.smooth_v)
             oh.copy_(od, non_blocking=True)
 
         for _ in range(2):
@@ -333,7 +337,7 @@ def run_sage2(args, cfg, world, rank, local):
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ops, dt, desc = oracle_sample(cfg, q, k, v, args.cpu_blocks)
+        ops, dt, desc = oracle_sample(cfg, q, k, v, args.cpu_blocks, args.qk_bits, args.smooth_v)
         cpu = {"value": ops / dt / 1e12, "unit": "TOPS", "cores": blas_threads(),
                "kind": "oracle", "sample": desc, "seconds": dt}
 
@@ -342,10 +346,10 @@ def run_sage2(args, cfg, world, rank, local):
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8/e4m3 (INT4 values)",
+            "dtype": "int8/e4m3 (INT4 values)" if args.qk_bits == 4 else "int8/e4m3 (INT8 values)",
             "data": "synthetic (seeded; distributions of the workload)",
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
-                       "causal": cfg.causal, "input_dtype": cfg.dtype,
+                       "causal": cfg.causal, "input_dtype": cfg.dtype, "variant": variant,
                        "parallelism": f"replicas x{world} (independent heads, no collective)",
                        "l2": "inputs larger than L2 (3 x %d MB per step)" %
                              (q.numel() * q.element_size() // 2 ** 20)},
@@ -366,6 +370,9 @@ def main():
                     help="query blocks per step of the oracle in --impl reference")
     ap.add_argument("--cpu-blocks", type=int, default=48,
                     help="query blocks of the oracle sample behind cpu_baseline")
+    ap.add_argument("--qk-bits", type=int, default=4, choices=[4, 8],
+                    help="4: the method (INT4 Q/K); 8: the INT8 variant")
+    ap.add_argument("--smooth-v", action="store_true", help="the V-smoothing variant")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -192,6 +192,27 @@ sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int H, int N, int d, int dtype, int o_dtype, int causal,
                                     float sm_scale, sage2_stream_t stream);
 
+/*
+ * Variable-length (packed) sequences: the forward pass of sage2_attn_fwd_ex
+ * applied to each of S sequences packed along the token axis.  The method's
+ * package names such an entry ("sageattn_varlen", codewithpapers page, code
+ * samples list); the pages give no more, so each sequence is treated as its
+ * own batch element: it attends only within itself (causal: top-left inside
+ * the sequence) and gets its own K mean, Q block means, scales, correction and
+ * per-channel V scales.
+ *   q, k, v, o  : HEAD-MAJOR packed [H, T, d] (q/k/v in `dtype`, o in `o_dtype`);
+ *                 sequence s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1.
+ *   cu_seqlens  : HOST int32 array of S+1 offsets, cu_seqlens[0] = 0,
+ *                 non-decreasing, cu_seqlens[S] = T (empty sequences allowed).
+ * The library takes one workspace for the longest sequence (as sage2_attn_fwd)
+ * and runs the sequences one after another on `stream`.  Other arguments and
+ * statuses as sage2_attn_fwd_ex; a malformed cu_seqlens is SAGE2_ERR_INVALID_ARG.
+ */
+sage2_status sage2_attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                   const int* cu_seqlens, int S, int H, int T, int d, int dtype,
+                                   int o_dtype, int causal, float sm_scale, int qk_format,
+                                   int smooth_v, sage2_stream_t stream);
+
 /* Bytes of workspace sage2_attn_fwd takes for this problem (0 on bad sizes). */
 size_t sage2_workspace_bytes(int B, int H, int N, int d);
 

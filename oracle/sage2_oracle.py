@@ -441,3 +441,35 @@ def sage2_head(Q, K, V, causal: bool, sm_scale: float | None = None, q_blocks=No
         pay["v_t"], pay["v_scale"] = quant_v(V)
     O, amb, rows = attn_quantized(pay, N, causal, sm_scale, q_blocks=q_blocks)
     return pay, O, amb, rows
+
+
+# ----------------------------------------------------------------------------
+# Variable-length (packed) sequences.  The method's package names a varlen
+# entry ("sageattn_varlen", codewithpapers page, code samples list) and the
+# pages give no more.  Reading: each packed sequence is its own batch element:
+# attention within the sequence only, and every step above (means, scales,
+# correction, V scales) computed per sequence.
+# ----------------------------------------------------------------------------
+
+def sage2_varlen_head(Q, K, V, cu_seqlens, causal: bool, sm_scale: float | None = None,
+                      qk_bits: int = 4, smooth_v: bool = False):
+    """One head of packed sequences: Q, K, V [T, d]; cu_seqlens [S+1] offsets.
+    Returns (O [T, d] float64, amb [T, d] float64)."""
+    Q = np.asarray(Q, np.float32)
+    T, d = Q.shape
+    cu = [int(c) for c in cu_seqlens]
+    if cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must rise from 0 to T")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    O = np.zeros((T, d))
+    amb = np.zeros((T, d))
+    for a, b in zip(cu, cu[1:]):
+        if b == a:
+            continue
+        _, o, m, rows = sage2_head(Q[a:b], K[a:b], V[a:b], causal, sm_scale,
+                                   qk_bits=qk_bits, smooth_v=smooth_v)
+        O[a + rows] = o
+        amb[a + rows] = m
+    return O, amb
+

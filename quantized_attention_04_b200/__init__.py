@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "sage2_smooth_quant_qk", "sage2_quant_v", "sage2_attn_fwd_quantized", "sage2_attn_fwd",
-    "sage2_attn_fwd_noalloc", "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
+    "sage2_attn_fwd_noalloc", "sage2_attn_fwd_varlen", "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
     "sage2_status_string", "sage2_version", "attn", "Sage2Error", "lib", "LIB_PATH",
 ]
 
@@ -50,6 +50,7 @@ _SIGS = {
                                          _F, _I, _P]),
     "sage2_attn_fwd_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sage2_debug_qk_s32_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "sage2_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sage2_check_device_error": (_I, [_P]),
     "sage2_status_string": (ctypes.c_char_p, [_I]),
     "sage2_version": (_I, []),
@@ -236,6 +237,35 @@ def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bo
 
 
 attn = sage2_attn_fwd
+
+
+def sage2_attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens,
+                          causal: bool = False, sm_scale: float | None = None, out_dtype=None,
+                          out: torch.Tensor | None = None, qk_bits: int = 4,
+                          smooth_v: bool = False) -> torch.Tensor:
+    """Packed variable-length sequences: q, k, v head-major [H, T, d] CUDA
+    tensors, cu_seqlens the S+1 token offsets (host ints).  Each sequence is
+    attended within itself; returns o [H, T, d]."""
+    if qk_bits not in _QKF:
+        raise ValueError("qk_bits must be 4 or 8")
+    for t in (q, k, v):
+        if t.dim() != 3 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors [H, T, d]")
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k and v must have the same shape and dtype")
+    H, T, d = q.shape
+    cu = [int(c) for c in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    arr = (ctypes.c_int * len(cu))(*cu)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(H, T, d, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib().sage2_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), arr, len(cu) - 1, H, T,
+                                     d, _DT[q.dtype], _DT[out.dtype], int(bool(causal)),
+                                     float(sm_scale), _QKF[qk_bits], int(bool(smooth_v)),
+                                     _stream(q))
+    _check("sage2_attn_fwd_varlen", st)
+    return out
 
 
 def sage2_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,

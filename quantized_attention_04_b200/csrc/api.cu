@@ -170,6 +170,39 @@ static cudaMemPool_t device_pool(int dev) {
   return pools[dev];
 }
 
+// One forward pass over B*H heads of N tokens: q/k/v heads ldh tokens apart,
+// o heads ldo tokens apart, payloads in the workspace ws (layout(g)), all on st.
+static cudaError_t forward(const void* q, const void* k, const void* v, void* o, const Dims& g,
+                           int dtype, int o_dtype, int causal, float sm_scale, int qk_bits,
+                           int smooth_v, int64_t ldh, int64_t ldo, uint8_t* ws, cudaStream_t st) {
+  const int B = g.B, H = g.H, N = g.N, d = g.d;
+  const Workspace w = layout(g);
+  cudaError_t e;
+  uint8_t* q_i4 = reinterpret_cast<uint8_t*>(ws + w.off_q_i4);
+  uint8_t* k_i4 = reinterpret_cast<uint8_t*>(ws + w.off_k_i4);
+  uint8_t* vt = ws + w.off_vt;
+  float* qs = reinterpret_cast<float*>(ws + w.off_qs);
+  float* ks = reinterpret_cast<float*>(ws + w.off_ks);
+  float* qm = reinterpret_cast<float*>(ws + w.off_qm);
+  float* km = reinterpret_cast<float*>(ws + w.off_km);
+  float* corr = reinterpret_cast<float*>(ws + w.off_corr);
+  float* vs = reinterpret_cast<float*>(ws + w.off_vs);
+  float* part = reinterpret_cast<float*>(ws + w.off_part);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
+  float* vmean = smooth_v ? reinterpret_cast<float*>(ws + w.off_vmean) : nullptr;
+
+  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
+            ws + w.off_qsplit, causal, qk_bits, ldh};
+  // the V mean reuses the K-mean scratch: stream order puts it after the K mean
+  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, vmean, part, ldh};
+  AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
+              sm_scale, qk_bits, vmean, ldo};
+  e = launch_smooth_quant_qk(qa, st);
+  if (e == cudaSuccess) e = launch_quant_v(va, st);
+  if (e == cudaSuccess) e = launch_attn(aa, st);
+  return e;
+}
+
 }  // namespace sage2
 
 using namespace sage2;
@@ -202,7 +235,7 @@ sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, i
   if (e != cudaSuccess) return from_cuda(e);
   QKArgs a{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean,
            qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, 0,
-           qk_bits_of(qk_format)};
+           qk_bits_of(qk_format), static_cast<int64_t>(N)};
   e = launch_smooth_quant_qk(a, st);
   const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
@@ -240,7 +273,8 @@ sage2_status sage2_quant_v_ex(const void* v, int dtype, int B, int H, int N, int
   if (e != cudaSuccess) return from_cuda(e);
   VArgs a{v, dtype, B, H, N, d, g.Np, g.NB, v_fp8_t, v_scale,
           reinterpret_cast<uint32_t*>(scratch), v_mean,
-          v_mean ? reinterpret_cast<float*>(scratch + amax_bytes) : nullptr};
+          v_mean ? reinterpret_cast<float*>(scratch + amax_bytes) : nullptr,
+          static_cast<int64_t>(N)};
   e = launch_quant_v(a, st);
   const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
@@ -269,7 +303,7 @@ sage2_status sage2_attn_fwd_quantized_ex(const uint8_t* q_i4, const float* q_sca
   if (s != SAGE2_OK) return s;
   AttnArgs a{q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale, o, o_dtype,
              B,    H,       N,    d,       g.Np,    g.NB,    causal,  sm_scale,
-             qk_bits_of(qk_format), v_mean};
+             qk_bits_of(qk_format), v_mean, static_cast<int64_t>(N)};
   return from_cuda(launch_attn(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -316,29 +350,8 @@ sage2_status sage2_attn_fwd_ex(const void* q, const void* k, const void* v, void
   e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), w.total, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
 
-  uint8_t* q_i4 = reinterpret_cast<uint8_t*>(ws + w.off_q_i4);
-  uint8_t* k_i4 = reinterpret_cast<uint8_t*>(ws + w.off_k_i4);
-  uint8_t* vt = ws + w.off_vt;
-  float* qs = reinterpret_cast<float*>(ws + w.off_qs);
-  float* ks = reinterpret_cast<float*>(ws + w.off_ks);
-  float* qm = reinterpret_cast<float*>(ws + w.off_qm);
-  float* km = reinterpret_cast<float*>(ws + w.off_km);
-  float* corr = reinterpret_cast<float*>(ws + w.off_corr);
-  float* vs = reinterpret_cast<float*>(ws + w.off_vs);
-  float* part = reinterpret_cast<float*>(ws + w.off_part);
-  uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
-  float* vmean = smooth_v ? reinterpret_cast<float*>(ws + w.off_vmean) : nullptr;
-  const int qk_bits = qk_bits_of(qk_format);
-
-  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
-            ws + w.off_qsplit, causal, qk_bits};
-  // the V mean reuses the K-mean scratch: stream order puts it after the K mean
-  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, vmean, part};
-  AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
-              sm_scale, qk_bits, vmean};
-  e = launch_smooth_quant_qk(qa, st);
-  if (e == cudaSuccess) e = launch_quant_v(va, st);
-  if (e == cudaSuccess) e = launch_attn(aa, st);
+  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, qk_bits_of(qk_format), smooth_v,
+              static_cast<int64_t>(N), static_cast<int64_t>(N), ws, st);
   const cudaError_t e2 = cudaFreeAsync(ws, st);
   return from_cuda(e != cudaSuccess ? e : e2);
 }

@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                const float* __restrict__ k_scale, const float* __restrict__ qk_corr,
                const float* __restrict__ v_scale, const float* __restrict__ v_mean,
-               void* __restrict__ out, int N, int Np, int NB, int causal, float L) {
+               void* __restrict__ out, int N, long long ldo, int Np, int NB, int causal,
+               float L) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -512,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = mbar_wait_warp(&sm.l_full, 0, abort_flag);
     if (ok && row < N) {
       const float inv = 1.0f / sm.lsum[r];
-      const size_t obase = (static_cast<size_t>(bh) * N + row) * D;
+      const size_t obase = (static_cast<size_t>(bh) * ldo + row) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 8) {
         float f[8];
@@ -547,8 +548,8 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const float L = a.sm_scale * 1.4426950408889634f;
   k_attn_fwd<D, OT, QB><<<dim3(a.NB, BH), kThreads, smem, st>>>(
-      tq, tk, tv, a.q_scale, a.k_scale, a.qk_corr, a.v_scale, a.v_mean, a.o, a.N, a.Np, a.NB,
-      a.causal, L);
+      tq, tk, tv, a.q_scale, a.k_scale, a.qk_corr, a.v_scale, a.v_mean, a.o, a.N, a.ldo, a.Np,
+      a.NB, a.causal, L);
   return cudaGetLastError();
 }
 

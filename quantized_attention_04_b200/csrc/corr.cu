@@ -246,7 +246,7 @@ cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st) {
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.N),
                               static_cast<uint64_t>(BH)};
     const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2,
-                                 static_cast<uint64_t>(a.N) * D * 2};
+                                 static_cast<uint64_t>(a.ldh) * D * 2};
     const uint32_t box[3] = {64, 128, 1};
     cudaError_t e = make_tmap(&tmk, a.k, 3, dims, strides, box, 2, 128);
     if (e != cudaSuccess) return e;

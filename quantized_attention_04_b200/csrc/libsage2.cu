@@ -7,3 +7,4 @@
 #include "attn.cu"
 #include "api.cu"
 #include "noalloc.cu"
+#include "varlen.cu"

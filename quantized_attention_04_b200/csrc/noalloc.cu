@@ -86,25 +86,7 @@ extern "C" sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, con
   if (ws == nullptr) return SAGE2_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-  uint8_t* q_i4 = reinterpret_cast<uint8_t*>(ws + w.off_q_i4);
-  uint8_t* k_i4 = reinterpret_cast<uint8_t*>(ws + w.off_k_i4);
-  uint8_t* vt = ws + w.off_vt;
-  float* qs = reinterpret_cast<float*>(ws + w.off_qs);
-  float* ks = reinterpret_cast<float*>(ws + w.off_ks);
-  float* qm = reinterpret_cast<float*>(ws + w.off_qm);
-  float* km = reinterpret_cast<float*>(ws + w.off_km);
-  float* corr = reinterpret_cast<float*>(ws + w.off_corr);
-  float* vs = reinterpret_cast<float*>(ws + w.off_vs);
-  float* part = reinterpret_cast<float*>(ws + w.off_part);
-  uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
-
-  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
-            ws + w.off_qsplit, causal, 4};
-  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, nullptr, nullptr};  // amax is cleared on the stream
-  AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
-              sm_scale, 4, nullptr};
-  e = launch_smooth_quant_qk(qa, st);
-  if (e == cudaSuccess) e = launch_quant_v(va, st);
-  if (e == cudaSuccess) e = launch_attn(aa, st);
+  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, 4, 0, static_cast<int64_t>(N),
+              static_cast<int64_t>(N), ws, st);
   return from_cuda(e);
 }

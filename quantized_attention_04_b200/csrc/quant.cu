@@ -55,7 +55,8 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162flo
 // chunk sums its chunk token by token in ascending order (fp32).
 // grid (ceil(nchunks / workers_per_block), B*H), 256 threads.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) k_mean_partial(const T* __restrict__ k, int N, int nchunks,
+__global__ void __launch_bounds__(256) k_mean_partial(const T* __restrict__ k, int N,
+                                                      long long ldh, int nchunks,
                                                       float* __restrict__ part) {
   constexpr int TPR = D / 8;
   constexpr int WPB = 256 / TPR;
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(256) k_mean_partial(const T* __restrict__ k, i
   if (chunk >= nchunks) return;
   const int t0 = chunk * 128;
   const int nt = min(128, N - t0);
-  const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bh * N + t0) * D) + q8;
+  const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bh * ldh + t0) * D) + q8;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -109,7 +110,7 @@ __global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int
 // computing its mean), z = 1 the K block (after subtracting kbar).  256 threads.
 template <typename T, int D, bool Q8>
 __global__ void __launch_bounds__(256) k_smooth_quant(
-    const T* __restrict__ q, const T* __restrict__ k, int N, int Np, int NB,
+    const T* __restrict__ q, const T* __restrict__ k, int N, long long ldh, int Np, int NB,
     const float* __restrict__ kmean, uint8_t* __restrict__ q_i4, float* __restrict__ q_scale,
     float* __restrict__ q_mean, uint8_t* __restrict__ k_i4, float* __restrict__ k_scale) {
   __shared__ __align__(16) T tile[128][D];
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
 
   // coalesced 16-byte loads of the valid rows
   constexpr int VPR = D / 8;  // uint4 per row
-  const uint4* g = reinterpret_cast<const uint4*>(src + ((size_t)bh * N + r0) * D);
+  const uint4* g = reinterpret_cast<const uint4*>(src + ((size_t)bh * ldh + r0) * D);
   uint4* s = reinterpret_cast<uint4*>(&tile[0][0]);
   for (int i = threadIdx.x; i < nvalid * VPR; i += 256) s[i] = __ldg(g + i);
 
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
 // threads; one 128-token chunk per block; float bits of |x| >= 0 are ordered
 // like unsigned integers, so atomicMax on the bits is exact.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
+__global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N, long long ldh,
                                                 const float* __restrict__ vmean,
                                                 uint32_t* __restrict__ amax_bits) {
   constexpr int TPR = D / 8;
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
     m[i] = 0.f;
     mu[i] = vmean ? vmean[(size_t)bh * D + q8 * 8 + i] : 0.f;   // V smoothing: |V - vbar|
   }
-  const uint4* src = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + t0) * D) + q8;
+  const uint4* src = reinterpret_cast<const uint4*>(v + ((size_t)bh * ldh + t0) * D) + q8;
   for (int t = r; t < nt; t += RPB) {
     float x[8];
     unpack8<T>(__ldg(src + (size_t)t * TPR), x);
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N,
 // grid (Np/128, B*H), 256 threads.  A warp owns one 16-token group and 32
 // consecutive channels, so its shared-memory reads are conflict-free.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N, int Np,
+__global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N, long long ldh, int Np,
                                                  const float* __restrict__ vmean,
                                                  const uint32_t* __restrict__ amax_bits,
                                                  uint8_t* __restrict__ vt,
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
   const int t0 = kt * 128;
   const int nvalid = max(0, min(128, N - t0));
   constexpr int VPR = D / 8;
-  const uint4* g = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + t0) * D);
+  const uint4* g = reinterpret_cast<const uint4*>(v + ((size_t)bh * ldh + t0) * D);
   uint4* s = reinterpret_cast<uint4*>(&tile[0][0]);
   for (int i = threadIdx.x; i < nvalid * VPR; i += 256) s[i] = __ldg(g + i);
   if (threadIdx.x < D) {
@@ -294,15 +295,15 @@ static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
   const int nchunks = a.NB;
   constexpr int WPB = 256 / (D / 8);
   k_mean_partial<T, D><<<dim3((nchunks + WPB - 1) / WPB, BH), 256, 0, st>>>(
-      static_cast<const T*>(a.k), a.N, nchunks, a.mean_part);
+      static_cast<const T*>(a.k), a.N, a.ldh, nchunks, a.mean_part);
   k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, nchunks, a.N, D, a.k_mean);
   if (a.qk_bits == 8)
     k_smooth_quant<T, D, true><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
         a.q_scale, a.q_mean, a.k_i4, a.k_scale);
   else
     k_smooth_quant<T, D, false><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.Np, a.NB, a.k_mean, a.q_i4,
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
         a.q_scale, a.q_mean, a.k_i4, a.k_scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -323,12 +324,12 @@ static cudaError_t launch_v_t(const VArgs& a, cudaStream_t st) {
     // V smoothing: the per-channel token mean, with the fixed order of the K mean
     constexpr int WPB = 256 / (D / 8);
     k_mean_partial<T, D><<<dim3((a.NB + WPB - 1) / WPB, BH), 256, 0, st>>>(
-        static_cast<const T*>(a.v), a.N, a.NB, a.mean_part);
+        static_cast<const T*>(a.v), a.N, a.ldh, a.NB, a.mean_part);
     k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, a.NB, a.N, D, a.v_mean);
   }
-  k_v_amax<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.v_mean,
+  k_v_amax<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.ldh, a.v_mean,
                                                  a.amax_bits);
-  k_v_quant<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.Np,
+  k_v_quant<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.ldh, a.Np,
                                                   a.v_mean, a.amax_bits, a.v_fp8_t, a.v_scale);
   return cudaGetLastError();
 }

@@ -24,6 +24,7 @@ struct QKArgs {
   void* qbar_split;        // scratch [3][B*H][NBc*128][d] in the input dtype (NBc = ceil(NB/128))
   int skip_masked_corr;    // 1: skip correction blocks a causal mask hides
   int qk_bits;             // 4: INT4 values as e4m3 codes; 8: INT8 values (two's complement)
+  int64_t ldh;             // tokens between consecutive heads of q and k (N when contiguous)
 };
 
 struct VArgs {
@@ -35,6 +36,7 @@ struct VArgs {
   uint32_t* amax_bits;     // scratch [B*H, d]
   float* v_mean;           // nullptr: no V smoothing; else the per-channel token mean [B*H, d]
   float* mean_part;        // scratch [B*H, NB, d] for the V mean (when v_mean is set)
+  int64_t ldh;             // tokens between consecutive heads of v (N when contiguous)
 };
 
 struct AttnArgs {
@@ -52,6 +54,7 @@ struct AttnArgs {
   float sm_scale;
   int qk_bits;             // 4 or 8 (payload format, see QKArgs)
   const float* v_mean;     // nullptr: V was not smoothed
+  int64_t ldo;             // tokens between consecutive heads of o (N when contiguous)
 };
 
 cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st);

@@ -32,7 +32,9 @@ def test_header_declares_the_boundary():
                  "sage2_check_device_error", "sage2_status_string",
                  # the variants (INT8 Q/K, V smoothing)
                  "sage2_attn_fwd_ex", "sage2_smooth_quant_qk_ex", "sage2_quant_v_ex",
-                 "sage2_attn_fwd_quantized_ex", "sage2_debug_qk_s32_ex"):
+                 "sage2_attn_fwd_quantized_ex", "sage2_debug_qk_s32_ex",
+                 # packed variable-length sequences
+                 "sage2_attn_fwd_varlen"):
         assert must in names
 
 
@@ -109,6 +111,28 @@ def test_validation_variant_entries(L):
                                          None) == 3
     assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 7, P, None) == 1
     assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 1, 0, None) == 1
+
+
+def test_validation_varlen(L):
+    import ctypes
+    def call(cu, S=None, H=2, T=None, d=64, **kw):
+        arr = (ctypes.c_int * len(cu))(*cu)
+        S = len(cu) - 1 if S is None else S
+        T = cu[-1] if T is None else T
+        a = dict(q=P, k=P, v=P, o=P, dt=0, odt=2, causal=0, sm=0.125, fmt=0, smooth=0)
+        a.update(kw)
+        return L.sage2_attn_fwd_varlen(a["q"], a["k"], a["v"], a["o"], arr, S, H, T, d, a["dt"],
+                                       a["odt"], a["causal"], a["sm"], a["fmt"], a["smooth"], None)
+    assert call([1, 5, 9]) == 1            # must start at 0
+    assert call([0, 5, 3]) == 1            # must not decrease
+    assert call([0, 5, 9], T=10) == 1      # must end at T
+    assert call([0, 5, 9], S=0) == 1
+    assert call([0, 5, 9], d=96) == 2
+    assert call([0, 5, 9], fmt=4) == 1
+    assert call([0, 5, 9], smooth=3) == 1
+    assert call([0, 5, 9], q=P + 8) == 3
+    assert call([0, 5, 9], causal=2) == 1
+    assert L.sage2_attn_fwd_varlen(P, P, P, P, None, 2, 2, 9, 64, 0, 2, 0, 0.1, 0, 0, None) == 1
 
 
 def test_workspace_bytes(L):

@@ -142,3 +142,43 @@ def test_v_smoothing_helps_offset_v():
         _, O, _, _ = orc.sage2_head(Q, K, V, False, sm, qk_bits=8, smooth_v=sv)
         err[sv] = np.abs(O - ref).mean()
     assert err[True] < 0.5 * err[False]
+
+
+# ------------------------------------------------------- packed sequences
+def test_varlen_equal_lengths_equal_batched_heads():
+    """Equal-length packed sequences are exactly the batched fixed-length path,
+    one sequence per batch element."""
+    rng = np.random.default_rng(17)
+    S, N, d = 3, 130, 32
+    Q = rng.standard_normal((S * N, d)).astype(np.float32)
+    K = (rng.standard_normal((S * N, d)) * 2).astype(np.float32)
+    V = rng.standard_normal((S * N, d)).astype(np.float32)
+    sm = 1 / math.sqrt(d)
+    for causal in (False, True):
+        O, amb = orc.sage2_varlen_head(Q, K, V, [0, N, 2 * N, 3 * N], causal, sm)
+        for s in range(S):
+            sl = slice(s * N, (s + 1) * N)
+            _, o, m, rows = orc.sage2_head(Q[sl], K[sl], V[sl], causal, sm)
+            assert np.array_equal(O[sl][rows], o) and np.array_equal(amb[sl][rows], m)
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    """Changing one sequence leaves the others' outputs bit-identical, and an
+    empty sequence is allowed."""
+    rng = np.random.default_rng(18)
+    d = 32
+    cu = [0, 5, 5, 200, 329]
+    T = cu[-1]
+    Q = rng.standard_normal((T, d)).astype(np.float32)
+    K = rng.standard_normal((T, d)).astype(np.float32)
+    V = rng.standard_normal((T, d)).astype(np.float32)
+    O1, _ = orc.sage2_varlen_head(Q, K, V, cu, True)
+    K2 = K.copy()
+    K2[200:] += 5
+    V2 = V.copy()
+    V2[200:] *= 3
+    O2, _ = orc.sage2_varlen_head(Q, K2, V2, cu, True)
+    assert np.array_equal(O1[:200], O2[:200])
+    assert not np.array_equal(O1[200:], O2[200:])
+    with pytest.raises(ValueError):
+        orc.sage2_varlen_head(Q, K, V, [0, 10, 5, T], True)
