@@ -359,6 +359,79 @@ def run_sage2(args, cfg, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- packed sequences
+def varlen_lengths(S: int):
+    """The packed workload: S causal bf16 sequences, H=32, d=128, with seeded
+    lengths uniform on [256, 4096] (a serving-style mix)."""
+    rng = np.random.default_rng(2000 + S)
+    return [int(x) for x in rng.integers(256, 4097, S)]
+
+
+def run_varlen(args, world, rank, local):
+    import quantized_attention_04_b200 as qa
+    from quantized_attention_04_b200.inputs import Config, Dist
+    lens = varlen_lengths(args.varlen)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(int).tolist()
+    T, H, d = cu[-1], 32, 128
+    cfg = Config(f"VL{args.varlen}", 1, H, T, d, True, "bf16",
+                 q=Dist(2.0), k=Dist(2.0, outliers=4, outlier_scale=20.0),
+                 v=Dist(2.0, outliers=4, outlier_scale=20.0), index=40 + args.varlen)
+    q, k, v = (t[0] for t in make_qkv(cfg))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    od = torch.empty_like(qd)
+    sm = 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        qa.sage2_attn_fwd_varlen(qd, kd, vd, cu, causal=True, sm_scale=sm, out=od,
+                                 qk_bits=args.qk_bits, smooth_v=args.smooth_v)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if qa.sage2_check_device_error(dev) != 0:
+        raise RuntimeError("device error during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world)
+    ops = sum(4.0 * H * n * n * d / 2 for n in lens) * world
+    value = ops / (ms * 1e-3) / 1e12
+    bf16_peak, _, _, peak_src = load_peaks()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8/e4m3 (INT4 values)" if args.qk_bits == 4 else "int8/e4m3 (INT8 values)",
+            "data": "synthetic (seeded; distributions of the workload)",
+            "config": {"workload": cfg.name, "sequences": len(lens), "tokens": T, "H": H, "d": d,
+                       "causal": True, "input_dtype": "bf16", "lengths": lens,
+                       "variant": ("int4" if args.qk_bits == 4 else "int8")
+                                  + ("+smooth_v" if args.smooth_v else ""),
+                       "parallelism": f"replicas x{world} (independent heads, no collective)"},
+            # one C call runs every kernel of every sequence: the whole step is measured
+            "roofline": {"bound": "tensor", "achieved": value, "peak": 2.0 * bf16_peak,
+                         "unit": "TFLOP/s", "frac": value / (2.0 * bf16_peak), "traffic": None,
+                         "kernel": "whole varlen step (all kernels, every sequence)",
+                         "peak_source": f"{peak_src} bf16 burst x 2"},
+            "cpu_baseline": None, "e2e": None, "clocks": clk.summary(),
+            # per sequence: K mean (2), smoothing+INT4, q-mean split, correction, V amax,
+            # V quant, attention; V smoothing adds the V mean (2)
+            "gpu_launches": (10 if args.smooth_v else 8) * sum(1 for n in lens if n) * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -373,6 +446,8 @@ def main():
     ap.add_argument("--qk-bits", type=int, default=4, choices=[4, 8],
                     help="4: the method (INT4 Q/K); 8: the INT8 variant")
     ap.add_argument("--smooth-v", action="store_true", help="the V-smoothing variant")
+    ap.add_argument("--varlen", type=int, default=0,
+                    help="time the packed-sequence entry on this many seeded sequences instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -384,7 +459,10 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_sage2(args, cfg, world, rank, local)
+        if args.varlen:
+            run_varlen(args, world, rank, local)
+        else:
+            run_sage2(args, cfg, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
