@@ -25,7 +25,7 @@
 //   warps 12-15   correction warpgroup: thread r owns query row r and the outer
 //                 fp32 accumulator (acc = alpha*acc + inner per key tile: the
 //                 outer level of the two-level accumulation), then the epilogue.
-// TMEM columns: S[b] at 128*b (b = 0, 1), inner[b] at 256 + d*b.
+// TMEM columns: S[b] at 128*b (b = 0, 1, 2), the inner accumulator at 384.
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout the kernel
 // records it in the device error word and every role leaves its loop.
 #include <cuda.h>
@@ -39,6 +39,7 @@
 namespace sage2 {
 
 constexpr int kStages = 4;
+constexpr int kSBuf = 3;                         // S tiles in flight (TMEM) and P~ tiles (smem)
 constexpr int kThreads = 512;
 constexpr int kSegStride = 36;                   // floats between the 32-key groups in shared memory
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
@@ -50,7 +51,7 @@ struct __align__(1024) AttnSmem {
   uint8_t q[128 * D];              // Q^ tile (K-major, swizzled)
   uint8_t k[kStages][128 * D];     // K^ tiles
   uint8_t v[kStages][D * 128];     // V^T tiles: D rows (channels) x 128 tokens
-  uint8_t p[2][128 * 128];         // P~ tiles: 128 rows x 128 tokens (e4m3)
+  uint8_t p[kSBuf][128 * 128];     // P~ tiles: 128 rows x 128 tokens (e4m3)
   // qk_corr and k_scale of the key tile: keys 32g..32g+31 at [36g, 36g+32).
   // The 16-byte gaps put the four groups (read by the four threads g of a
   // row in the same instruction) in different banks.
@@ -63,14 +64,14 @@ struct __align__(1024) AttnSmem {
   float lsum[128];                  // final row sums (448-scaled), softmax -> correction
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2];               // two arrivals: the MMA thread once it saw the key
+  uint64_t s_full[kSBuf];               // two arrivals: the MMA thread once it saw the key
                                     // tile land (so its scales are visible to whoever
                                     // acquires this barrier), and the commit of S[b]
-  uint64_t p_full[2];               // P~[b] written by all 8 softmax warps; this also
+  uint64_t p_full[kSBuf];               // P~[b] written by all 8 softmax warps; this also
                                     // says S[b] was read and inner[b] of tile t-2 folded
-  uint64_t i_full[2];               // two arrivals: the MMA thread after it saw p_full (so
-                                    // alpha of the tile is visible), and the commit of inner[b]
-  uint64_t i_empty[2];              // the correction warpgroup read inner[b]
+  uint64_t i_full;                  // two arrivals: the MMA thread after it saw p_full (so
+                                    // alpha of the tile is visible), and the commit of inner
+  uint64_t i_empty;                 // the correction warpgroup read inner
   uint64_t l_full;                  // the softmax warps published the row sums
   uint64_t drain;
   uint32_t tmem_base;
@@ -249,12 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSBuf; ++b) {
       mbar_init(&sm.s_full[b], 2);
       mbar_init(&sm.p_full[b], 8);
-      mbar_init(&sm.i_full[b], 2);
-      mbar_init(&sm.i_empty[b], 4);
     }
+    mbar_init(&sm.i_full, 2);
+    mbar_init(&sm.i_empty, 4);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.l_full, 8);
     sm.abort_flag = 0;
@@ -320,10 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kStageK = (128 * D) >> 4, kStageV = (D * 128) >> 4, kStageP = (128 * 128) >> 4;
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
       auto issue_qk = [&](int u) -> bool {
-        const int s = u % kStages, b = u & 1;
+        const int s = u % kStages, b = u % kSBuf;
         if (!mbar_wait(&sm.kv_full[s], (u / kStages) & 1, abort_flag)) return false;
         // S[b] is free once the softmax of tile u-2 is past its P~ store
-        if (u >= 2 && !mbar_wait(&sm.p_full[b], ((u >> 1) - 1) & 1, abort_flag)) return false;
+        if (u >= kSBuf && !mbar_wait(&sm.p_full[b], ((u / kSBuf) - 1) & 1, abort_flag)) return false;
         mbar_arrive(&sm.s_full[b]);                       // releases the kv_full acquire
         tc_fence_after();
         const uint64_t kb = dk + s * kStageK;
@@ -336,27 +337,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_pv = [&](int u) -> bool {
-        const int s = u % kStages, b = u & 1;
+        const int s = u % kStages, b = u % kSBuf;
         // P~(u) and alpha(u) are written; the correction warpgroup has read
-        // inner[b] of tile u-2
-        if (!mbar_wait(&sm.p_full[b], (u >> 1) & 1, abort_flag)) return false;
-        if (u >= 2 && !mbar_wait(&sm.i_empty[b], ((u >> 1) - 1) & 1, abort_flag)) return false;
-        mbar_arrive(&sm.i_full[b]);                       // releases the p_full acquire (alpha)
+        // inner of tile u-1 (one inner accumulator: it is read well before the
+        // next PV is due)
+        if (!mbar_wait(&sm.p_full[b], (u / kSBuf) & 1, abort_flag)) return false;
+        if (u >= 1 && !mbar_wait(&sm.i_empty, (u - 1) & 1, abort_flag)) return false;
+        mbar_arrive(&sm.i_full);                          // releases the p_full acquire (alpha)
         tc_fence_after();
         const uint64_t pb = dp + b * kStageP, vb = dv + s * kStageV;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + 256 + b * D, pb + 2 * kk, vb + 2 * kk, idesc_pv, kk > 0);
-        tc_commit(&sm.i_full[b]);
+        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + kSBuf * 128, pb + 2 * kk, vb + 2 * kk, idesc_pv, kk > 0);
+        tc_commit(&sm.i_full);
         tc_commit(&sm.kv_empty[s]);
         return true;
       };
-      if (ok) ok = issue_qk(0);
-      if (ok && nt > 1) ok = issue_qk(1);
+      for (int u = 0; ok && u < kSBuf && u < nt; ++u) ok = issue_qk(u);
       for (int t = 0; ok && t < nt; ++t) {
         // both wait for the end of the softmax of tile t; PV first, its result
-        // is needed one tile earlier than S(t+2)
+        // is needed before S(t+3)
         if (!issue_pv(t)) { ok = false; break; }
-        if (t + 2 < nt && !issue_qk(t + 2)) { ok = false; break; }
+        if (t + kSBuf < nt && !issue_qk(t + kSBuf)) { ok = false; break; }
       }
       if (!ok) {
         // wait for every MMA issued so far before the block frees TMEM
@@ -397,11 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bar_other = (h == 0 ? kBarExpB : kBarExpA) + quad;
 
     for (int t = 0; t < nt; ++t) {
-      const int s = t % kStages, b = t & 1;
-      // s_full(t) also says PV(t-2) is complete: the MMA thread issued QK(t)
-      // after PV(t-2), and the commit tracks every earlier MMA.  So P~[b] is
+      const int s = t % kStages, b = t % kSBuf;
+      // s_full(t) also says PV(t-3) is complete: the MMA thread issued QK(t)
+      // after PV(t-3), and the commit tracks every earlier MMA.  So P~[b] is
       // free, with no wait of its own.
-      if (ok) ok = mbar_wait_warp(&sm.s_full[b], (t >> 1) & 1, abort_flag);
+      if (ok) ok = mbar_wait_warp(&sm.s_full[b], (t / kSBuf) & 1, abort_flag);
       if (!ok) {
         if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
         named_bar_arrive(bar_other, 64);
@@ -437,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
       const float2 alpha = make_float2(ex2((m0 - mn0) * L), ex2((m1 - mn1) * L));  // 0 on the first tile
       // for the correction warpgroup; slot t%4 was last read for tile t-4,
-      // before PV(t-2) was issued, which s_full(t) follows
+      // before PV(t-3) was issued, which s_full(t) follows
       sm.alpha[t & 3][r0] = alpha.x;                      // the row's four threads agree
       sm.alpha[t & 3][r0 + 8] = alpha.y;
       // p448 = 448 * exp2((x' - m) L) = exp2(x' L - (m L - log2 448))
@@ -446,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // exp2 turn: the first warpgroup waits for the second one's previous tile,
       // the second one for the first one's current tile
       if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
-      // the P~ buffer of this parity is free: PV(t-2) completed (see s_full above)
+      // the P~ buffer b is free: PV(t-3) completed (see s_full above)
       uint8_t* p0 = sm.p[b] + r0 * 128;
       uint8_t* p1 = p0 + 8 * 128;
       const float s0 = exp_pack_store(x0, L2, nb0, p0, g, r0 & 7);
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_inc<168>();
     const int r = (warp & 3) * 32 + lane;
     const int row = qt * 128 + r;
-    const uint32_t tI = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + 256;
+    const uint32_t tI = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kSBuf * 128;
     for (int i = r; i < D; i += 128) {
       sm.vsc[i] = v_scale[static_cast<size_t>(bh) * D + i];
       sm.vmean[i] = v_mean ? v_mean[static_cast<size_t>(bh) * D + i] : 0.f;
@@ -493,22 +494,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < D; ++c) acc[c] = 0.f;
     bool ok = true;
     for (int t = 0; ok && t < nt; ++t) {
-      const int b = t & 1;
       // i_full also carries the MMA thread's release after it saw p_full, so
       // alpha of tile t is visible
-      if (!mbar_wait_warp(&sm.i_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&sm.i_full, t & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const float al = sm.alpha[t & 3][r];
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tI + b * D + c0, v);
+        tmem_ld32(tI + c0, v);
         tmem_ld_wait();
         fold32(acc + c0, v, al);
       }
       tc_fence_before();
       __syncwarp();
-      mbar_arrive_lane0(&sm.i_empty[b], lane);
+      mbar_arrive_lane0(&sm.i_empty, lane);
     }
     if (ok) ok = mbar_wait_warp(&sm.l_full, 0, abort_flag);
     if (ok && row < N) {
