@@ -16,9 +16,12 @@
 // k_qbar_split : qbar -> three 16-bit terms, [3][B*H][NBc*128][d] (pad rows 0).
 // k_qk_corr_tc : one CTA = one head, one 128-block chunk, a run of key tiles.
 //   warp 0 TMA (the chunk's three term tiles once, then K tiles, 2 stages),
-//   warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 epilogue (thread =
-//   block row; writes 128 consecutive keys of C per tile).  TMA zero-fills
-//   keys >= N, so their C is 0.
+//   warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 epilogue: a warp owns
+//   32 block rows; per tile it stages four 32 x 32 fp32 boxes in shared memory
+//   (128-byte swizzle, conflict-free) and writes each with a TMA tensor store,
+//   so C leaves in full lines (one thread per row writing its own row would
+//   scatter every warp store over 32 rows).  TMA zero-fills keys >= N on the
+//   load side, so their C is 0; the store clips block rows >= NB.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <climits>
@@ -75,6 +78,7 @@ template <int D>
 struct __align__(1024) CorrSmem {
   uint8_t a[3][D / 64][128 * 128];   // term x 128-byte atom x (128 rows x 128 B)
   uint8_t b[2][D / 64][128 * 128];   // stage x atom: 128 keys x 64 channels
+  uint8_t out[4][2][32 * 128];       // epilogue warp x buffer: 32 rows x 32 fp32 (swizzled)
   uint64_t a_full;
   uint64_t b_full[2], b_empty[2];
   uint64_t d_full[2], d_empty[2];
@@ -86,8 +90,8 @@ struct __align__(1024) CorrSmem {
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 1)
     k_qk_corr_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_k,
-                 int N, int Np, int NB, int NBc, int BH, int skip_masked,
-                 float* __restrict__ corr) {
+                 const __grid_constant__ CUtensorMap tm_c, int N, int Np, int NB, int NBc,
+                 int BH, int skip_masked) {
   extern __shared__ uint8_t smem_raw[];
   CorrSmem<D>& sm = *reinterpret_cast<CorrSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -183,39 +187,46 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp >= 4) {
-    // epilogue: thread = block row of the chunk, 128 keys per tile
+    // epilogue: warp q owns block rows 32q..32q+31 of the chunk (its TMEM lanes)
     const int q = warp - 4;
-    const int blk = chunk * 128 + q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    float* crow = corr + (static_cast<size_t>(bh) * NB + (blk < NB ? blk : 0)) * Np;
+    const int row0 = chunk * 128 + q * 32;
+    int nb = 0;                                          // staging buffer to fill next
     for (int i = 0; i < ntiles; ++i) {
       const int s = i & 1;
       if (!mbar_wait_warp(&sm.d_full[s], (i >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      uint32_t v0[32], v1[32], v2[32], v3[32];
-      tmem_ld32(tmem + s * 128 + lane_off + 0, v0);
-      tmem_ld32(tmem + s * 128 + lane_off + 32, v1);
-      tmem_ld32(tmem + s * 128 + lane_off + 64, v2);
-      tmem_ld32(tmem + s * 128 + lane_off + 96, v3);
+      uint32_t v[4][32];
+      tmem_ld32(tmem + s * 128 + lane_off + 0, v[0]);
+      tmem_ld32(tmem + s * 128 + lane_off + 32, v[1]);
+      tmem_ld32(tmem + s * 128 + lane_off + 64, v[2]);
+      tmem_ld32(tmem + s * 128 + lane_off + 96, v[3]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.d_empty[s]);
-      if (blk < NB) {
-        float4* dst = reinterpret_cast<float4*>(crow + (kt0 + i) * 128);
+      mbar_arrive_lane0(&sm.d_empty[s], lane);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          dst[c] = make_float4(__uint_as_float(v0[4 * c]), __uint_as_float(v0[4 * c + 1]),
-                               __uint_as_float(v0[4 * c + 2]), __uint_as_float(v0[4 * c + 3]));
-          dst[8 + c] = make_float4(__uint_as_float(v1[4 * c]), __uint_as_float(v1[4 * c + 1]),
-                                   __uint_as_float(v1[4 * c + 2]), __uint_as_float(v1[4 * c + 3]));
-          dst[16 + c] = make_float4(__uint_as_float(v2[4 * c]), __uint_as_float(v2[4 * c + 1]),
-                                    __uint_as_float(v2[4 * c + 2]), __uint_as_float(v2[4 * c + 3]));
-          dst[24 + c] = make_float4(__uint_as_float(v3[4 * c]), __uint_as_float(v3[4 * c + 1]),
-                                    __uint_as_float(v3[4 * c + 2]), __uint_as_float(v3[4 * c + 3]));
+      for (int grp = 0; grp < 4; ++grp) {
+        // the store issued two boxes ago has finished reading this buffer
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint8_t* st = sm.out[q][nb];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(st + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(v[grp][4 * c], v[grp][4 * c + 1], v[grp][4 * c + 2], v[grp][4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_c, st, (kt0 + i) * 128 + 32 * grp, row0, bh);
+          bulk_commit();
         }
+        nb ^= 1;
       }
     }
+    // shared memory stays in use until the last stores have read it
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -251,6 +262,17 @@ cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st) {
     cudaError_t e = make_tmap(&tmk, a.k, 3, dims, strides, box, 2, 128);
     if (e != cudaSuccess) return e;
   }
+  alignas(64) CUtensorMap tmc;
+  {
+    // C as [B*H][NB][Np] fp32; a box is 32 keys (128 B, swizzled) x 32 block rows
+    const uint64_t dims[3] = {static_cast<uint64_t>(a.Np), static_cast<uint64_t>(a.NB),
+                              static_cast<uint64_t>(BH)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.Np) * 4,
+                                 static_cast<uint64_t>(a.NB) * a.Np * 4};
+    const uint32_t box[3] = {32, 32, 1};
+    cudaError_t e = make_tmap(&tmc, a.qk_corr, 3, dims, strides, box, 4, 128);
+    if (e != cudaSuccess) return e;
+  }
   const size_t smem = sizeof(CorrSmem<D>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_qk_corr_tc<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -258,7 +280,7 @@ cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int groups = (a.NB + kCorrTilesPerCta - 1) / kCorrTilesPerCta;
   k_qk_corr_tc<T, D><<<dim3(groups, NBc, BH), 256, smem, st>>>(
-      tma, tmk, a.N, a.Np, a.NB, NBc, BH, a.skip_masked_corr, a.qk_corr);
+      tma, tmk, tmc, a.N, a.Np, a.NB, NBc, BH, a.skip_masked_corr);
   return cudaGetLastError();
 }
 
