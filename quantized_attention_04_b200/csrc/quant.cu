@@ -150,29 +150,62 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   // .16x256b TMEM loads then give each thread 32 consecutive keys).  Q^ rows
   // keep their natural order.
   constexpr int CPL = D / 32;  // channels per lane: 4 (D=128) or 2 (D=64)
+  constexpr float kQmax = Q8 ? 127.f : 7.f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < 128; r += 8) {
-    float x[CPL];
-    float amax = 0.f;
+  float mu[CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      const int c = lane * CPL + i;
-      x[i] = (r < nvalid) ? __fsub_rn(to_f32(tile[r][c]), mean[c]) : 0.f;
-      amax = fmaxf(amax, fabsf(x[i]));
+  for (int i = 0; i < CPL; ++i) mu[i] = mean[lane * CPL + i];
+  // this lane's CPL consecutive channels of row r, smoothed (one 4- or 8-byte load)
+  auto load_row = [&](int r, float (&x)[CPL]) {
+    float raw[CPL];
+    if (CPL == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(&tile[r][lane * 4]);
+      const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) raw[i] = to_f32(h[i]);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(&tile[r][lane * 2]);
+      const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) raw[i] = to_f32(h[i]);
     }
 #pragma unroll
+    for (int i = 0; i < CPL; ++i) x[i] = (r < nvalid) ? __fsub_rn(raw[i], mu[i]) : 0.f;
+  };
+  // The warp owns rows warp + 8j, j = 0..15.  Pass 1: every row's amax; lane j
+  // keeps row j's, so that the two IEEE divisions of all 16 rows take one
+  // instruction sequence of the warp instead of sixteen.
+  float my_amax = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < 16; ++j) {
+    float x[CPL];
+    load_row(warp + 8 * j, x);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    // INT4 (the method): each value in [-7, 7] is stored as its e4m3 code:
-    // every such integer is exact in e4m3, so the FP8 tensor path multiplies
-    // the INT4 values exactly (at the same rate as the 8-bit integer path) and
-    // yields S as an fp32 integer.  Zero is stored as +0 (code 0x00).
-    // INT8 (the variant): values in [-127, 127] as two's-complement bytes.
-    constexpr float kQmax = Q8 ? 127.f : 7.f;
+    my_amax = lane == j ? amax : my_amax;
+  }
+  const bool nz = my_amax > 0.f;
+  const float my_sc = nz ? __fdiv_rn(my_amax, kQmax) : 0.f;
+  const float my_inv = nz ? __fdiv_rn(kQmax, my_amax) : 0.f;
+  // Pass 2: quantize with row j's inverse scale (from lane j).
+  // INT4 (the method): each value in [-7, 7] is stored as its e4m3 code:
+  // every such integer is exact in e4m3, so the FP8 tensor path multiplies
+  // the INT4 values exactly (at the same rate as the 8-bit integer path) and
+  // yields S as an fp32 integer.  Zero is stored as +0 (code 0x00).
+  // INT8 (the variant): values in [-127, 127] as two's-complement bytes.
+#pragma unroll 4
+  for (int j = 0; j < 16; ++j) {
+    const int r = warp + 8 * j;
+    const float inv = __shfl_sync(0xffffffffu, my_inv, j);
+    const float sc = __shfl_sync(0xffffffffu, my_sc, j);
+    const bool row_nz = __shfl_sync(0xffffffffu, my_amax, j) > 0.f;   // sc may underflow to 0
+    float x[CPL];
+    load_row(r, x);
     uint32_t packed = 0;
-    float sc = 0.f;
-    if (amax > 0.f) {
-      sc = __fdiv_rn(amax, kQmax);
-      const float inv = __fdiv_rn(kQmax, amax);
+    if (row_nz) {
 #pragma unroll
       for (int i = 0; i < CPL; ++i) {
         float v = rintf(__fmul_rn(x[i], inv));
