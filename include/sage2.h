@@ -238,6 +238,15 @@ sage2_status sage2_debug_qk_s32_ex(const uint8_t* q_i4, const uint8_t* k_i4, int
                                    int d, int qk_format, int32_t* s_out, sage2_stream_t stream);
 
 /*
+ * Test entry for failure detection: launches one thread that waits on an
+ * mbarrier phase nothing completes.  The wait is bounded (about one second):
+ * it gives up, sets the device error word (SAGE2_ERR_TIMEOUT on the next
+ * sage2_check_device_error) and the kernel returns normally, so the context
+ * stays usable.  Every wait of the library's kernels behaves the same way.
+ */
+sage2_status sage2_debug_wait_timeout(sage2_stream_t stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the device error word that
  * kernels set instead of trapping.  SAGE2_ERR_TIMEOUT if a bounded wait ran
  * out, SAGE2_ERR_CUDA on a sticky CUDA error, else SAGE2_OK.

@@ -52,6 +52,7 @@ _SIGS = {
     "sage2_debug_qk_s32_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "sage2_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sage2_check_device_error": (_I, [_P]),
+    "sage2_debug_wait_timeout": (_I, [_P]),
     "sage2_status_string": (ctypes.c_char_p, [_I]),
     "sage2_version": (_I, []),
 }
@@ -301,3 +302,11 @@ def sage2_debug_qk_s32(q_i4: torch.Tensor, k_i4: torch.Tensor, N: int) -> torch.
                                      _QKF[_qk_bits_of(q_i4)], _ptr(s), _stream(q_i4))
     _check("sage2_debug_qk_s32_ex", st)
     return s
+
+
+def sage2_debug_wait_timeout(device=None) -> None:
+    """Failure-detection test entry: a kernel whose bounded wait runs out
+    (see include/sage2.h).  sage2_check_device_error() then reports 6."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check("sage2_debug_wait_timeout", lib().sage2_debug_wait_timeout(st))

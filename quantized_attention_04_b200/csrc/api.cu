@@ -382,6 +382,10 @@ sage2_status sage2_debug_qk_s32(const uint8_t* q_i4, const uint8_t* k_i4, int B,
   return sage2_debug_qk_s32_ex(q_i4, k_i4, B, H, N, d, SAGE2_QK_INT4, s_out, stream);
 }
 
+sage2_status sage2_debug_wait_timeout(sage2_stream_t stream) {
+  return from_cuda(launch_debug_wait_timeout(reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sage2_status sage2_check_device_error(sage2_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return SAGE2_ERR_CUDA;

@@ -111,3 +111,22 @@ cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int
 }
 
 }  // namespace sage2
+
+// Test kernel for failure detection: one thread waits on an mbarrier phase
+// that nothing completes.  The bounded wait gives up after its limit, records
+// the timeout in the device error word and returns; the kernel ends normally
+// and the context stays usable (no trap, no fault).
+namespace sage2 {
+__global__ void k_debug_wait_timeout() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, nullptr);   // phase 0 never completes: times out
+  }
+}
+cudaError_t launch_debug_wait_timeout(cudaStream_t st) {
+  k_debug_wait_timeout<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
+}
+}  // namespace sage2

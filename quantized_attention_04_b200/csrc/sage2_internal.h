@@ -60,6 +60,7 @@ struct AttnArgs {
 cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_debug_wait_timeout(cudaStream_t st);
 cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int Np, int d,
                             int qk_bits, int32_t* s_out, cudaStream_t st);
 
