@@ -8,7 +8,8 @@ FP8 V, the fused attention kernel) over one batch of the workload, through the
 C ABI's three stage calls (sage2_smooth_quant_qk, sage2_quant_v,
 sage2_attn_fwd_quantized: the kernels sage2_attn_fwd runs, into caller-owned
 payload buffers), with CUDA events around each attention launch; the e2e leg
-calls sage2_attn_fwd itself with host buffers copied in and out every step.  The default workload is the causal bf16 prefill case
+calls sage2_attn_fwd_host with pinned host buffers: every step copies the
+inputs in and the output back (pipelined by heads inside the call).  The default workload is the causal bf16 prefill case
 B=1, H=32, N=32768, d=128 (the long-sequence d=128 point at which the tensor
 roofline target is stated).  Metric: TOPS = 4*B*H*N^2*d / t, halved for causal.
 Under torchrun each rank runs its own full copy of the workload (heads are
@@ -309,13 +310,11 @@ def run_sage2(args, cfg, world, rank, local):
         qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
         oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
 
+        # the public host-buffer entry: chunks of heads are copied in, run and
+        # copied back on library streams, overlapping copies with kernels
         def e2e_step():
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out=od,
-                              qk_bits=args.qk_bits, smooth_v=args.smooth_v)
-            oh.copy_(od, non_blocking=True)
+            qa.sage2_attn_fwd_host(qh, kh, vh, oh, causal=cfg.causal, sm_scale=sm,
+                                   qk_bits=args.qk_bits, smooth_v=args.smooth_v, device=dev)
 
         for _ in range(2):
             e2e_step()

@@ -217,6 +217,23 @@ sage2_status sage2_attn_fwd_varlen(const void* q, const void* k, const void* v, 
                                    int o_dtype, int causal, float sm_scale, int qk_format,
                                    int smooth_v, sage2_stream_t stream);
 
+/*
+ * The forward pass of sage2_attn_fwd_ex over HOST tensors: q, k, v, o are host
+ * pointers ([B,H,N,d] as sage2_attn_fwd), PINNED (cudaHostAlloc /
+ * cudaHostRegister) for the copies to overlap; other host memory still works,
+ * with the copies serialised by the driver.  Whole heads are copied in, run
+ * and copied back in chunks (about 96 MB of inputs each) on up to three
+ * library streams forked from and joined back into `stream`, so the copies of
+ * some chunks overlap the kernels of others.  Device buffers for the chunks in
+ * flight come from the library's pool.  The call returns once everything is
+ * enqueued: o is complete when `stream` reaches that point.  Statuses as
+ * sage2_attn_fwd_ex (pointers are only checked for NULL).
+ */
+sage2_status sage2_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int B,
+                                 int H, int N, int d, int dtype, int o_dtype, int causal,
+                                 float sm_scale, int qk_format, int smooth_v,
+                                 sage2_stream_t stream);
+
 /* Bytes of workspace sage2_attn_fwd takes for this problem (0 on bad sizes). */
 size_t sage2_workspace_bytes(int B, int H, int N, int d);
 

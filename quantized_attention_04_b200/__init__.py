@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "sage2_smooth_quant_qk", "sage2_quant_v", "sage2_attn_fwd_quantized", "sage2_attn_fwd",
-    "sage2_attn_fwd_noalloc", "sage2_attn_fwd_varlen", "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
+    "sage2_attn_fwd_noalloc", "sage2_attn_fwd_varlen", "sage2_attn_fwd_host", "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
     "sage2_status_string", "sage2_version", "attn", "Sage2Error", "lib", "LIB_PATH",
 ]
 
@@ -53,6 +53,7 @@ _SIGS = {
     "sage2_attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sage2_check_device_error": (_I, [_P]),
     "sage2_debug_wait_timeout": (_I, [_P]),
+    "sage2_attn_fwd_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sage2_status_string": (ctypes.c_char_p, [_I]),
     "sage2_version": (_I, []),
 }
@@ -310,3 +311,31 @@ def sage2_debug_wait_timeout(device=None) -> None:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     _check("sage2_debug_wait_timeout", lib().sage2_debug_wait_timeout(st))
+
+
+def sage2_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                        causal: bool = False, sm_scale: float | None = None, qk_bits: int = 4,
+                        smooth_v: bool = False, device=None) -> torch.Tensor:
+    """The forward pass over HOST tensors [B,H,N,d] (pinned for overlap): chunks of
+    heads are copied in, run and copied back on library streams joined into the
+    current stream of `device`; `out` (host) is complete once that stream is."""
+    if qk_bits not in _QKF:
+        raise ValueError("qk_bits must be 4 or 8")
+    for t in (q, k, v, out):
+        if t.dim() != 4 or t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, out must be contiguous host tensors [B, H, N, d]")
+    for t in (k, v):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k and v must have the same shape and dtype")
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    B, H, N, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    status = lib().sage2_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
+                                       _DT[q.dtype], _DT[out.dtype], int(bool(causal)),
+                                       float(sm_scale), _QKF[qk_bits], int(bool(smooth_v)), st)
+    _check("sage2_attn_fwd_host", status)
+    return out

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsage2.so")
 SOURCES = ["libsage2.cu"]  # includes the files below (one translation unit)
-HEADERS = ["api.cu", "quant.cu", "attn.cu", "debug_qk.cu", "noalloc.cu", "varlen.cu", "corr.cu", "sm100_ptx.cuh", "sage2_internal.h"]
+HEADERS = ["api.cu", "quant.cu", "attn.cu", "debug_qk.cu", "noalloc.cu", "varlen.cu", "host_pipe.cu", "corr.cu", "sm100_ptx.cuh", "sage2_internal.h"]
 
 
 def nvcc_path() -> str:

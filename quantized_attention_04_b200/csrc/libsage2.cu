@@ -8,3 +8,4 @@
 #include "api.cu"
 #include "noalloc.cu"
 #include "varlen.cu"
+#include "host_pipe.cu"
