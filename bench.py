@@ -37,7 +37,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from quantized_attention_04_b200.inputs import CONFIGS, make_qkv  # noqa: E402
+from quantized_attention_04_b200.inputs import CONFIGS, make_qkv, sweep_config  # noqa: E402
 
 METRIC = "quantized attention TOPS (4*B*H*N^2*d/t, halved if causal)"
 KERNELS_PER_STEP = 8   # k_mean_partial, k_mean_finalize, k_smooth_quant, k_qbar_split, k_qk_corr_tc,
@@ -117,16 +117,21 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- dist
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None, timeout_s: float = 120.0):
+    """One process per GPU (torchrun's env): NCCL on GPUs, gloo without (the
+    CPU tests of this plumbing).  Returns (world, rank, local_rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return world, rank, local
 
 
@@ -137,12 +142,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: every multi-GPU number is the max over ranks."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(ops_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job throughput (TOPS): every rank runs its own copy of the
+    workload (weak scaling), timed by the slowest rank."""
+    return ops_per_rank * world / (ms * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- recorded DRAM traffic
@@ -290,7 +303,7 @@ def run_sage2(args, cfg, world, rank, local):
     ms = max_over_ranks(ms_local, world)
     clocks = clk.summary()
     total_ops = cfg.ops() * world
-    value = total_ops / (ms * 1e-3) / 1e12
+    value = aggregate(cfg.ops(), ms, world)
 
     # ---- dominant kernel: its average launch inside the timed region
     attn_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in attn_ev), world)
@@ -431,6 +444,73 @@ def run_varlen(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- roofline sweep
+def run_sweep(args, world, rank, local):
+    """The causal bf16 sweep d in {64, 128} x N in {4096, 16384, 32768} at B=1,
+    H=32: per point, the whole step and the attention launch (CUDA events around
+    it inside the timed steps), one JSON line each."""
+    import quantized_attention_04_b200 as qa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    bf16_peak, _, _, peak_src = load_peaks()
+    for d in (64, 128):
+        for N in (4096, 16384, 32768):
+            cfg = sweep_config(N, d)
+            q, k, v = make_qkv(cfg)
+            qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+            od = torch.empty_like(qd)
+            sm = 1.0 / math.sqrt(d)
+            stream = torch.cuda.current_stream(dev)
+            pay = qa.sage2_smooth_quant_qk(qd, kd)
+            vpay = qa.sage2_quant_v(vd)
+            attn_ev = []
+
+            def step(record):
+                qa.sage2_smooth_quant_qk(qd, kd, out=pay)
+                qa.sage2_quant_v(vd, out=vpay)
+                if record:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                qa.sage2_attn_fwd_quantized(pay, vpay[0], vpay[1], N, True, sm, out=od)
+                if record:
+                    e1.record(stream)
+                    attn_ev.append((e0, e1))
+
+            for _ in range(args.warmup):
+                step(False)
+            torch.cuda.synchronize()
+            barrier(world)
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(local) as clk:
+                ev0.record(stream)
+                for _ in range(args.steps):
+                    step(True)
+                ev1.record(stream)
+                torch.cuda.synchronize()
+            barrier(world)
+            if qa.sage2_check_device_error(dev) != 0:
+                raise RuntimeError("device error in the sweep")
+            ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world)
+            attn_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in attn_ev), world)
+            ops = cfg.ops()
+            if rank == 0:
+                print(json.dumps({
+                    "metric": METRIC, "value": ops * world / (ms * 1e-3) / 1e12, "unit": "TOPS",
+                    "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                    "dtype": "int8/e4m3 (INT4 values)", "data": "synthetic (seeded; LLM-like)",
+                    "config": {"workload": cfg.name, "B": 1, "H": 32, "N": N, "d": d,
+                               "causal": True, "input_dtype": "bf16"},
+                    "roofline": {"bound": "tensor", "achieved": ops / (attn_ms * 1e-3) / 1e12,
+                                 "peak": 2.0 * bf16_peak, "unit": "TFLOP/s",
+                                 "frac": ops / (attn_ms * 1e-3) / 1e12 / (2.0 * bf16_peak),
+                                 "traffic": None, "kernel": "k_attn_fwd", "kernel_ms": attn_ms,
+                                 "peak_source": f"{peak_src} bf16 burst x 2"},
+                    "clocks": clk.summary(), "gpu_launches": KERNELS_PER_STEP * args.steps,
+                }), flush=True)
+            del qd, kd, vd, od, pay, vpay
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -445,6 +525,8 @@ def main():
     ap.add_argument("--qk-bits", type=int, default=4, choices=[4, 8],
                     help="4: the method (INT4 Q/K); 8: the INT8 variant")
     ap.add_argument("--smooth-v", action="store_true", help="the V-smoothing variant")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the causal bf16 sweep d x N at B=1, H=32 (one line per point)")
     ap.add_argument("--varlen", type=int, default=0,
                     help="time the packed-sequence entry on this many seeded sequences instead")
     ap.add_argument("--no-e2e", action="store_true")
@@ -458,7 +540,9 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        if args.varlen:
+        if args.sweep:
+            run_sweep(args, world, rank, local)
+        elif args.varlen:
             run_varlen(args, world, rank, local)
         else:
             run_sage2(args, cfg, world, rank, local)
