@@ -206,16 +206,23 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
     load_row(r, x);
     uint32_t packed = 0;
     if (row_nz) {
+      // |x| <= amax and inv = RN(qmax/amax), so |x*inv| <= qmax*(1+2^-24)^2 <
+      // qmax + 1/2: the rounded value never leaves [-qmax, qmax] and needs no
+      // clamp.  Adding +0 turns a rounded -0 into +0 (the oracle's integer 0).
+      float v[CPL];
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        float v = rintf(__fmul_rn(x[i], inv));
-        v = fminf(fmaxf(v, -kQmax), kQmax);
-        const int vi = static_cast<int>(v);                          // -0 -> 0
-        const uint32_t byte =
-            Q8 ? (static_cast<uint32_t>(vi) & 0xFFu)
-               : static_cast<uint32_t>(__nv_cvt_float_to_fp8(static_cast<float>(vi),
-                                                              __NV_SATFINITE, __NV_E4M3));
-        packed |= byte << (8 * i);
+      for (int i = 0; i < CPL; ++i) v[i] = __fadd_rn(rintf(__fmul_rn(x[i], inv)), 0.f);
+      if (Q8) {
+#pragma unroll
+        for (int i = 0; i < CPL; ++i)
+          packed |= (static_cast<uint32_t>(static_cast<int>(v[i])) & 0xFFu) << (8 * i);
+      } else {
+        // exact e4m3 codes of the integers, two per conversion
+#pragma unroll
+        for (int i = 0; i < CPL; i += 2)
+          packed |= static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(v[i], v[i + 1]),
+                                                                     __NV_SATFINITE, __NV_E4M3))
+                    << (8 * i);
       }
     }
     const int srow = is_q ? r : 8 * ((r >> 1) & 15) + 2 * (r >> 5) + (r & 1);
