@@ -9,9 +9,11 @@
 //                 the key scales and the correction chunk (kStages-deep ring).
 //   warp 1        MMA issuer (one thread): S = Q^ K^T with tcgen05 kind::f8f6f4
 //                 (the INT4 values carried as e4m3 codes; exact fp32 integer
-//                 sums) into TMEM (two buffers, issued two key tiles ahead), and
-//                 inner = P~ V~ with kind::f8f6f4 (e4m3 -> f32) into a fresh
-//                 TMEM accumulator per key tile (two buffers).
+//                 sums; kind::i8 for the INT8 variant) into TMEM (three
+//                 buffers, issued three key tiles ahead), and inner = P~ V~
+//                 with kind::f8f6f4 (e4m3 -> f32) into a fresh TMEM
+//                 accumulator per key tile (one buffer: the correction
+//                 warpgroup reads it long before the next PV).
 //   warp 2        TMEM allocator.
 //   warps 4-7,    two softmax warpgroups.  Warpgroup h owns lanes 16h..16h+15 of
 //   warps 8-11    every 32-lane TMEM quadrant; with .16x256b loads a thread owns
@@ -68,7 +70,7 @@ struct __align__(1024) AttnSmem {
                                     // tile land (so its scales are visible to whoever
                                     // acquires this barrier), and the commit of S[b]
   uint64_t p_full[kSBuf];               // P~[b] written by all 8 softmax warps; this also
-                                    // says S[b] was read and inner[b] of tile t-2 folded
+                                    // says S[b] was read
   uint64_t i_full;                  // two arrivals: the MMA thread after it saw p_full (so
                                     // alpha of the tile is visible), and the commit of inner
   uint64_t i_empty;                 // the correction warpgroup read inner
