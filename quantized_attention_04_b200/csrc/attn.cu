@@ -125,13 +125,13 @@ __device__ __forceinline__ float2 s_pair(uint32_t a, uint32_t b) {
 // Dequantise + correct the 16 keys 4m..4m+3 (m = 0..3) of both rows held in
 // one .16x256b.x8 load: x' = sq_i * (sk_j * S_ij) + C_j.
 template <int QB>
-__device__ __forceinline__ void dequant16(const uint32_t (&sr)[32], const float* ck,
-                                          const float* kk, float2 a0, float2 a1, float* x0,
+__device__ __forceinline__ void dequant16(const uint32_t (&sr)[32], const float4* ck,
+                                          const float4* kk, float2 a0, float2 a1, float* x0,
                                           float* x1) {
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    const float4 c4 = *reinterpret_cast<const float4*>(ck + 4 * m);
-    const float4 k4 = *reinterpret_cast<const float4*>(kk + 4 * m);
+    const float4 c4 = ck[m];
+    const float4 k4 = kk[m];
     const float2 kxy = make_float2(k4.x, k4.y), kzw = make_float2(k4.z, k4.w);
     const float2 cxy = make_float2(c4.x, c4.y), czw = make_float2(c4.z, c4.w);
     const uint32_t* q = sr + 8 * m;
@@ -416,13 +416,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sA[32], sB[32];
         tmem_ld16x256_32(tS + b * 128, sA);
         tmem_ld16x256_32(tS + b * 128 + 64, sB);
-        tmem_ld_wait();
         // the key scales and correction chunk of stage s are visible: s_full
-        // also carries the MMA thread's release after it acquired kv_full
-        const float* ck = sm.corr[s] + kSegStride * g;
-        const float* kk = sm.ksc[s] + kSegStride * g;
-        dequant16<QB>(sA, ck, kk, a02, a12, x0, x1);
-        dequant16<QB>(sB, ck + 16, kk + 16, a02, a12, x0 + 16, x1 + 16);
+        // also carries the MMA thread's release after it acquired kv_full.
+        // The first half is read while the TMEM loads are in flight.
+        const float4* cp = reinterpret_cast<const float4*>(sm.corr[s] + kSegStride * g);
+        const float4* kp = reinterpret_cast<const float4*>(sm.ksc[s] + kSegStride * g);
+        float4 c0[4], k0[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          c0[m] = cp[m];
+          k0[m] = kp[m];
+        }
+        tmem_ld_wait();
+        dequant16<QB>(sA, c0, k0, a02, a12, x0, x1);
+        dequant16<QB>(sB, cp + 4, kp + 4, a02, a12, x0 + 16, x1 + 16);
       }
       if ((causal && t == qt) || (tail && t == NB - 1)) {
 #pragma unroll

@@ -106,7 +106,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                volatile int* abort_flag) {
   // fast path: the phase has completed (the common case in a pipelined loop);
   // the vote makes the branch warp-uniform
-  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  if (__all_sync(0xffffffffu, mbar_test(bar, parity))) return true;
   const bool ok = mbar_wait(bar, parity, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
