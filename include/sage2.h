@@ -38,7 +38,11 @@
  *  k_scale f32  [B,H,Np]     per-token scale
  *  k_mean f32   [B,H,d]      token mean of K
  *  qk_corr f32  [B,H,NB,Np]  q_mean[blk] . K[j] (raw K), 0 for j >= N
- *  v_fp8_t u8   [B,H,d,Np]   e4m3 codes of V * 448/amax_c, TRANSPOSED (token-contiguous)
+ *  v_fp8_t u8   [B,H,d,Np]   e4m3 codes of V * 448/amax_c, TRANSPOSED (token-contiguous).
+ *                            Tokens are PERMUTED inside each 128-token block: byte p of
+ *                            a block holds token sigma(p), where sigma swaps the 2-bit
+ *                            fields [6:5] and [4:3] of p (sigma = sigma^-1), i.e.
+ *                            sigma(p) = 32*((p/8)%4) + 8*((p/32)%4) + p%8.
  *  v_scale f32  [B,H,d]      per-channel scale amax_c/448
  */
 #ifndef SAGE2_H_
@@ -107,7 +111,8 @@ sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, i
 /*
  * FP8 e4m3 quantization of V with one scale per channel (Abstract: FP8 V).
  *   v        : [B,H,N,d] in `dtype`.
- *   v_fp8_t  : [B,H,d,Np] e4m3 codes, token-contiguous; pad tokens are 0.
+ *   v_fp8_t  : [B,H,d,Np] e4m3 codes, token-contiguous in the permuted order
+ *              of each 128-token block given above; pad tokens are 0.
  *   v_scale  : [B,H,d] = amax_c/448 (0 for an all-zero channel).
  * Codes are RNE of fp32(V * (448/amax_c)) with saturation to +-448.
  */

@@ -28,6 +28,8 @@
 //                 fp32 accumulator (acc = alpha*acc + inner per key tile: the
 //                 outer level of the two-level accumulation), then the epilogue.
 // TMEM columns: S[b] at 128*b (b = 0, 1, 2), the inner accumulator at 384.
+// P~ of a tile replaces the first 32 columns of its S buffer (its 128 keys as
+// bytes, four per column) and is the TMEM A operand of the PV product.
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout the kernel
 // records it in the device error word and every role leaves its loop.
 #include <cuda.h>
@@ -53,7 +55,6 @@ struct __align__(1024) AttnSmem {
   uint8_t q[128 * D];              // Q^ tile (K-major, swizzled)
   uint8_t k[kStages][128 * D];     // K^ tiles
   uint8_t v[kStages][D * 128];     // V^T tiles: D rows (channels) x 128 tokens
-  uint8_t p[kSBuf][128 * 128];     // P~ tiles: 128 rows x 128 tokens (e4m3)
   // qk_corr and k_scale of the key tile: keys 32g..32g+31 at [36g, 36g+32).
   // The 16-byte gaps put the four groups (read by the four threads g of a
   // row in the same instruction) in different banks.
@@ -69,6 +70,7 @@ struct __align__(1024) AttnSmem {
   uint64_t s_full[kSBuf];               // two arrivals: the MMA thread once it saw the key
                                     // tile land (so its scales are visible to whoever
                                     // acquires this barrier), and the commit of S[b]
+  uint64_t p_read[kSBuf];           // PV of the tile read its P~ out of S[b] (commit)
   uint64_t p_full[kSBuf];               // P~[b] written by all 8 softmax warps; this also
                                     // says S[b] was read
   uint64_t i_full;                  // two arrivals: the MMA thread after it saw p_full (so
@@ -160,16 +162,13 @@ __device__ __forceinline__ float rowmax32(const float (&x)[32]) {
 }
 
 // p448 = exp2(x' L + nb) for the 32 keys of one row, e4m3-rounded (RN,
-// saturating) and stored as two 16-byte chunks (keys 0-15, 16-31) of the
-// row's 128-byte line of P~: chunks 2g, 2g+1 of the line, XOR-swizzled by
-// `sw` (the row mod 8: the MMA's 128-byte swizzle).  Returns the row's sum
-// of the unrounded p448.
-__device__ __forceinline__ float exp_pack_store(const float (&x)[32], float2 L2, float2 nb,
-                                                uint8_t* prow, int g, int sw) {
+// saturating) into eight words: word i holds keys 4i..4i+3 (one byte each).
+// Returns the row's sum of the unrounded p448.
+__device__ __forceinline__ float exp_pack(const float (&x)[32], float2 L2, float2 nb,
+                                          uint32_t (&w)[8]) {
   float2 sumA = make_float2(0.f, 0.f), sumB = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    uint32_t w[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = c * 16 + u * 4;
@@ -183,9 +182,8 @@ __device__ __forceinline__ float exp_pack_store(const float (&x)[32], float2 L2,
       sumB = __fadd2_rn(sumB, e1);
       const uint32_t lo = __nv_cvt_float2_to_fp8x2(e0, __NV_SATFINITE, __NV_E4M3);
       const uint32_t hi = __nv_cvt_float2_to_fp8x2(e1, __NV_SATFINITE, __NV_E4M3);
-      w[u] = lo | (hi << 16);
+      w[4 * c + u] = lo | (hi << 16);
     }
-    *reinterpret_cast<uint4*>(prow + (((2 * g + c) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   const float2 s2 = __fadd2_rn(sumA, sumB);
   return s2.x + s2.y;
@@ -255,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < kSBuf; ++b) {
       mbar_init(&sm.s_full[b], 2);
       mbar_init(&sm.p_full[b], 8);
+      mbar_init(&sm.p_read[b], 1);
     }
     mbar_init(&sm.i_full, 2);
     mbar_init(&sm.i_empty, 4);
@@ -319,14 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq = smem_desc_kmajor(sm.q, D);
       const uint64_t dk = smem_desc_kmajor(sm.k[0], D);
       const uint64_t dv = smem_desc_kmajor(sm.v[0], 128);
-      const uint64_t dp = smem_desc_kmajor(sm.p[0], 128);
-      constexpr uint32_t kStageK = (128 * D) >> 4, kStageV = (D * 128) >> 4, kStageP = (128 * 128) >> 4;
+      constexpr uint32_t kStageK = (128 * D) >> 4, kStageV = (D * 128) >> 4;
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag);
       auto issue_qk = [&](int u) -> bool {
         const int s = u % kStages, b = u % kSBuf;
         if (!mbar_wait(&sm.kv_full[s], (u / kStages) & 1, abort_flag)) return false;
-        // S[b] is free once the softmax of tile u-2 is past its P~ store
-        if (u >= kSBuf && !mbar_wait(&sm.p_full[b], ((u / kSBuf) - 1) & 1, abort_flag)) return false;
+        // S[b] (with P~ of tile u-3 in its first 32 columns) is free once PV(u-3) read it
+        if (u >= kSBuf && !mbar_wait(&sm.p_read[b], ((u / kSBuf) - 1) & 1, abort_flag)) return false;
         mbar_arrive(&sm.s_full[b]);                       // releases the kv_full acquire
         tc_fence_after();
         const uint64_t kb = dk + s * kStageK;
@@ -347,11 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= 1 && !mbar_wait(&sm.i_empty, (u - 1) & 1, abort_flag)) return false;
         mbar_arrive(&sm.i_full);                          // releases the p_full acquire (alpha)
         tc_fence_after();
-        const uint64_t pb = dp + b * kStageP, vb = dv + s * kStageV;
+        const uint64_t vb = dv + s * kStageV;
+        // A = P~(u) in TMEM (the first 32 columns of S[b]: 128 keys, 4 per column)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + kSBuf * 128, pb + 2 * kk, vb + 2 * kk, idesc_pv, kk > 0);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ts(tmem + kSBuf * 128, tmem + b * 128 + 8 * kk, vb + 2 * kk, idesc_pv, kk > 0);
         tc_commit(&sm.i_full);
         tc_commit(&sm.kv_empty[s]);
+        tc_commit(&sm.p_read[b]);
         return true;
       };
       for (int u = 0; ok && u < kSBuf && u < nt; ++u) ok = issue_qk(u);
@@ -456,14 +457,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // exp2 turn: the first warpgroup waits for the second one's previous tile,
       // the second one for the first one's current tile
       if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
-      // the P~ buffer b is free: PV(t-3) completed (see s_full above)
-      uint8_t* p0 = sm.p[b] + r0 * 128;
-      uint8_t* p1 = p0 + 8 * 128;
-      const float s0 = exp_pack_store(x0, L2, nb0, p0, g, r0 & 7);
-      const float s1 = exp_pack_store(x1, L2, nb1, p1, g, r0 & 7);
+      // P~(t) goes to the first 32 columns of S[b], over scores this thread
+      // has already read: column 8k + 2g + e of its two rows holds its keys
+      // 32g + 8k + 4e .. +3 (V^T's tokens are stored in the matching order).
+      uint32_t w0[8], w1[8];
+      const float s0 = exp_pack(x0, L2, nb0, w0);
+      const float s1 = exp_pack(x1, L2, nb1, w1);
+      {
+        uint32_t pr[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            pr[4 * k + e] = w0[2 * k + e];
+            pr[4 * k + 2 + e] = w1[2 * k + e];
+          }
+        tmem_st16x256_16(tS + b * 128, pr);
+      }
       named_bar_arrive(bar_other, 64);
-      fence_proxy_async_smem();
-      tc_fence_before();                                  // S(t) reads are done
+      tmem_st_wait();
+      tc_fence_before();                                  // S(t) read, P~(t) written
       __syncwarp();
       mbar_arrive_lane0(&sm.p_full[b], lane);
       l0 = alpha.x * l0 + s0;

@@ -273,9 +273,13 @@ __global__ void __launch_bounds__(256) k_v_amax(const T* __restrict__ v, int N, 
   }
 }
 
-// V, pass 2: codes = e4m3_rn_satfinite(V * (448/amax_c)), stored transposed.
-// grid (Np/128, B*H), 256 threads.  A warp owns one 16-token group and 32
-// consecutive channels, so its shared-memory reads are conflict-free.
+// V, pass 2: codes = e4m3_rn_satfinite(V * (448/amax_c)), stored transposed
+// with the tokens of each 128-token block permuted: byte p of a channel's
+// block holds token sigma(p), sigma swapping the 2-bit fields [6:5] and [4:3]
+// of the index (an involution).  That is the key order in which the
+// attention kernel lays P~ out in tensor memory.
+// grid (Np/128, B*H), 256 threads.  A warp owns one 16-byte output group and
+// 32 consecutive channels, so its shared-memory reads are conflict-free.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N, long long ldh, int Np,
                                                  const float* __restrict__ vmean,
@@ -299,10 +303,10 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // work items: (channel group of 32, 16-token group): (D/32) * 8 items, 8 warps
+  // work items: (channel group of 32, 16-byte output group): (D/32) * 8 items, 8 warps
   for (int item = warp; item < (D / 32) * 8; item += 8) {
     const int c = (item / 8) * 32 + lane;
-    const int tg = item % 8;
+    const int og = item % 8;
     const float sc = inv[c], m0 = mu[c];
     uint32_t w[4];
 #pragma unroll
@@ -310,7 +314,9 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
       uint32_t word = 0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int r = tg * 16 + p * 4 + h * 2;
+        // bytes 16og + i, i = 4p + 2h + {0,1}: tokens sigma(16og + i), consecutive pairs
+        const int i = p * 4 + h * 2;
+        const int r = 32 * (((og & 1) << 1) | (i >> 3)) + 8 * (og >> 1) + (i & 7);
         const float x0 = (r < nvalid) ? __fmul_rn(__fsub_rn(to_f32(tile[r][c]), m0), sc) : 0.f;
         const float x1 = (r + 1 < nvalid) ? __fmul_rn(__fsub_rn(to_f32(tile[r + 1][c]), m0), sc) : 0.f;
         const __nv_fp8x2_storage_t two =
@@ -319,7 +325,7 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
       }
       w[p] = word;
     }
-    *reinterpret_cast<uint4*>(vt + ((size_t)bh * D + c) * Np + t0 + tg * 16) =
+    *reinterpret_cast<uint4*>(vt + ((size_t)bh * D + c) * Np + t0 + og * 16) =
         make_uint4(w[0], w[1], w[2], w[3]);
   }
 }

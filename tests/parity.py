@@ -101,5 +101,14 @@ def key_interleave(Np: int) -> np.ndarray:
     return blk * 128 + 32 * ((j // 2) % 4) + 2 * (j // 8) + j % 2
 
 
+def value_interleave(Np: int) -> np.ndarray:
+    """Index map of the library's permuted v_fp8_t token order: byte p of each
+    128-token block holds token sigma(p) of that block, sigma swapping the
+    2-bit fields [6:5] and [4:3] of p, so stored = natural[:, value_interleave(Np)]."""
+    n = np.arange(Np)
+    blk, j = n // 128, n % 128
+    return blk * 128 + 32 * ((j // 8) % 4) + 8 * ((j // 32) % 4) + j % 8
+
+
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)

@@ -97,6 +97,7 @@ def test_smoothed_v_payloads_bit_exact(qa, cfg):
         for h in range(cfg.H):
             ovt, ovs, ovm = orc.quant_v_smoothed(P.np32(v[b, h]))
             assert P.bits_equal(vm[b, h], ovm), ("v_mean", b, h)
+            ovt = ovt[:, P.value_interleave(ovt.shape[1])]    # the library's token order
             assert P.bits_equal(vt[b, h], ovt), ("v_fp8_t", b, h)
             assert P.bits_equal(vs[b, h], ovs), ("v_scale", b, h)
 
