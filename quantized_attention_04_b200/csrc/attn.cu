@@ -400,12 +400,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bar_mine = (h == 0 ? kBarExpA : kBarExpB) + quad;
     const int bar_other = (h == 0 ? kBarExpB : kBarExpA) + quad;
 
+    // s_full(t+1) is probed (non-blocking, with acquire) early in the exp2
+    // phase of tile t, so that the blocking wait is skipped when S(t+1) has
+    // landed by then: the probe's latency hides behind the exp2 work.
+    bool s_ready = false;
     for (int t = 0; t < nt; ++t) {
       const int s = t % kStages, b = t % kSBuf;
       // s_full(t) also says PV(t-3) is complete: the MMA thread issued QK(t)
       // after PV(t-3), and the commit tracks every earlier MMA.  So P~[b] is
       // free, with no wait of its own.
-      if (ok) ok = mbar_wait_warp(&sm.s_full[b], (t / kSBuf) & 1, abort_flag);
+      if (ok && !s_ready) ok = mbar_wait_warp(&sm.s_full[b], (t / kSBuf) & 1, abort_flag);
       if (!ok) {
         if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
         named_bar_arrive(bar_other, 64);
@@ -457,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // exp2 turn: the first warpgroup waits for the second one's previous tile,
       // the second one for the first one's current tile
       if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
+      const bool probe = t + 1 < nt && mbar_test(&sm.s_full[(t + 1) % kSBuf], ((t + 1) / kSBuf) & 1);
       // P~(t) goes to the first 32 columns of S[b], over scores this thread
       // has already read: column 8k + 2g + e of its two rows holds its keys
       // 32g + 8k + 4e .. +3 (V^T's tokens are stored in the matching order).
@@ -479,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();                                  // S(t) read, P~(t) written
       __syncwarp();
       mbar_arrive_lane0(&sm.p_full[b], lane);
+      s_ready = __all_sync(0xffffffffu, probe);           // the probe's result is consumed here
       l0 = alpha.x * l0 + s0;
       l1 = alpha.y * l1 + s1;
       m0 = mn0;
