@@ -11,9 +11,9 @@
 //                 (the INT4 values carried as e4m3 codes; exact fp32 integer
 //                 sums; kind::i8 for the INT8 variant) into TMEM (three
 //                 buffers, issued three key tiles ahead), and inner = P~ V~
-//                 with kind::f8f6f4 (e4m3 -> f32) into a fresh TMEM
-//                 accumulator per key tile (one buffer: the correction
-//                 warpgroup reads it long before the next PV).
+//                 with kind::f8f6f4 (e4m3 -> f32; A = P~ from TMEM) into a
+//                 fresh TMEM accumulator per key tile (one buffer: the
+//                 correction warpgroup reads it long before the next PV).
 //   warp 2        TMEM allocator.
 //   warps 4-7,    two softmax warpgroups.  Warpgroup h owns lanes 16h..16h+15 of
 //   warps 8-11    every 32-lane TMEM quadrant; with .16x256b loads a thread owns
@@ -21,9 +21,9 @@
 //                 threads of a warp share a row).  Per tile: dequantise +
 //                 correct its 64 scores, row max across the four threads, the
 //                 rescale factor alpha (to shared memory), exp2, l, and
-//                 P~ = e4m3(448 p) into shared memory (the MMA's swizzled
-//                 layout).  The exp2 phases of the two warps of a sub-partition
-//                 take turns (named barriers).
+//                 P~ = e4m3(448 p) into TMEM over the tile's S buffer.  The
+//                 exp2 phases of the two warps of a sub-partition take turns
+//                 (named barriers).
 //   warps 12-15   correction warpgroup: thread r owns query row r and the outer
 //                 fp32 accumulator (acc = alpha*acc + inner per key tile: the
 //                 outer level of the two-level accumulation), then the epilogue.
@@ -70,7 +70,6 @@ struct __align__(1024) AttnSmem {
   uint64_t s_full[kSBuf];               // two arrivals: the MMA thread once it saw the key
                                     // tile land (so its scales are visible to whoever
                                     // acquires this barrier), and the commit of S[b]
-  uint64_t p_read[kSBuf];           // PV of the tile read its P~ out of S[b] (commit)
   uint64_t p_full[kSBuf];               // P~[b] written by all 8 softmax warps; this also
                                     // says S[b] was read
   uint64_t i_full;                  // two arrivals: the MMA thread after it saw p_full (so
@@ -253,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < kSBuf; ++b) {
       mbar_init(&sm.s_full[b], 2);
       mbar_init(&sm.p_full[b], 8);
-      mbar_init(&sm.p_read[b], 1);
     }
     mbar_init(&sm.i_full, 2);
     mbar_init(&sm.i_empty, 4);
@@ -323,8 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_qk = [&](int u) -> bool {
         const int s = u % kStages, b = u % kSBuf;
         if (!mbar_wait(&sm.kv_full[s], (u / kStages) & 1, abort_flag)) return false;
-        // S[b] (with P~ of tile u-3 in its first 32 columns) is free once PV(u-3) read it
-        if (u >= kSBuf && !mbar_wait(&sm.p_read[b], ((u / kSBuf) - 1) & 1, abort_flag)) return false;
+        // S[b] (with P~ of tile u-3 in its first 32 columns) is free once PV(u-3)
+        // has completed: the phase of i_full for tile u-3 (QK(u) is issued right
+        // after PV(u-3), before PV(u-2), so i_full is still in that phase)
+        if (u >= kSBuf && !mbar_wait(&sm.i_full, (u - kSBuf) & 1, abort_flag)) return false;
         mbar_arrive(&sm.s_full[b]);                       // releases the kv_full acquire
         tc_fence_after();
         const uint64_t kb = dk + s * kStageK;
@@ -352,7 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f8_ts(tmem + kSBuf * 128, tmem + b * 128 + 8 * kk, vb + 2 * kk, idesc_pv, kk > 0);
         tc_commit(&sm.i_full);
         tc_commit(&sm.kv_empty[s]);
-        tc_commit(&sm.p_read[b]);
         return true;
       };
       for (int u = 0; ok && u < kSBuf && u < nt; ++u) ok = issue_qk(u);
