@@ -43,7 +43,7 @@
 namespace sage2 {
 
 constexpr int kStages = 4;
-constexpr int kSBuf = 3;                         // S tiles in flight (TMEM) and P~ tiles (smem)
+constexpr int kSBuf = 3;                         // S tiles in flight in TMEM (P~ of a tile over its S)
 constexpr int kThreads = 512;
 constexpr int kSegStride = 36;                   // floats between the 32-key groups in shared memory
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
@@ -67,10 +67,10 @@ struct __align__(1024) AttnSmem {
   float lsum[128];                  // final row sums (448-scaled), softmax -> correction
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[kSBuf];               // two arrivals: the MMA thread once it saw the key
+  uint64_t s_full[kSBuf];           // two arrivals: the MMA thread once it saw the key
                                     // tile land (so its scales are visible to whoever
                                     // acquires this barrier), and the commit of S[b]
-  uint64_t p_full[kSBuf];               // P~[b] written by all 8 softmax warps; this also
+  uint64_t p_full[kSBuf];           // P~ over S[b] written by all 8 softmax warps; this also
                                     // says S[b] was read
   uint64_t i_full;                  // two arrivals: the MMA thread after it saw p_full (so
                                     // alpha of the tile is visible), and the commit of inner
@@ -406,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < nt; ++t) {
       const int s = t % kStages, b = t % kSBuf;
       // s_full(t) also says PV(t-3) is complete: the MMA thread issued QK(t)
-      // after PV(t-3), and the commit tracks every earlier MMA.  So P~[b] is
-      // free, with no wait of its own.
+      // after PV(t-3) completed, and the commit tracks every earlier MMA.  So
+      // the P~ columns of S[b] are free, with no wait of its own.
       if (ok && !s_ready) ok = mbar_wait_warp(&sm.s_full[b], (t / kSBuf) & 1, abort_flag);
       if (!ok) {
         if (h == 1 || t > 0) named_bar_sync(bar_mine, 64);
