@@ -227,7 +227,7 @@ sage2_status sage2_attn_fwd_varlen(const void* q, const void* k, const void* v, 
  * pointers ([B,H,N,d] as sage2_attn_fwd), PINNED (cudaHostAlloc /
  * cudaHostRegister) for the copies to overlap; other host memory still works,
  * with the copies serialised by the driver.  Whole heads are copied in, run
- * and copied back in chunks (about 96 MB of inputs each) on up to three
+ * and copied back in chunks (about 48 MB of inputs each) on up to four
  * library streams forked from and joined back into `stream`, so the copies of
  * some chunks overlap the kernels of others.  Device buffers for the chunks in
  * flight come from the library's pool.  The call returns once everything is

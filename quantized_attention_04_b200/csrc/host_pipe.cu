@@ -16,8 +16,8 @@
 
 namespace sage2 {
 
-constexpr int kHostLanes = 3;
-constexpr size_t kHostChunkBytes = static_cast<size_t>(96) << 20;   // inputs per chunk (target)
+constexpr int kHostLanes = 4;
+constexpr size_t kHostChunkBytes = static_cast<size_t>(48) << 20;   // inputs per chunk (target)
 
 struct HostLanes {
   cudaStream_t s[kHostLanes] = {};
