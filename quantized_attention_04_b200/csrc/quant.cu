@@ -108,13 +108,21 @@ __global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int
 // ---------------------------------------------------------------------------
 // Smoothing + INT4.  grid (NB, B*H, 2): z = 0 quantizes the Q block (after
 // computing its mean), z = 1 the K block (after subtracting kbar).  256 threads.
+// Two lanes own one row (16 rows per warp), each half of its channels, so a
+// row's amax needs one shuffle and its scale none.  In shared memory row r
+// starts at byte RS*r and its second half at +HO (RS = 2D+32, HO = D+16): the
+// 16-byte chunks that the eight lanes of one access phase read then fall in
+// eight different bank groups.
 template <typename T, int D, bool Q8>
 __global__ void __launch_bounds__(256) k_smooth_quant(
     const T* __restrict__ q, const T* __restrict__ k, int N, long long ldh, int Np, int NB,
     const float* __restrict__ kmean, uint8_t* __restrict__ q_i4, float* __restrict__ q_scale,
     float* __restrict__ q_mean, uint8_t* __restrict__ k_i4, float* __restrict__ k_scale) {
-  __shared__ __align__(16) T tile[128][D];
-  __shared__ float mean[D];
+  constexpr int RS = 2 * D + 32, HO = D + 16;     // bytes
+  constexpr int CPR = D / 8, CPH = CPR / 2;       // 16-byte chunks per row / per half
+  constexpr int MH = D / 2 + 4;                   // floats between the two halves of mean
+  __shared__ __align__(16) uint8_t tile[128 * RS];
+  __shared__ __align__(16) float mean[2 * MH];
   const int blk = blockIdx.x, bh = blockIdx.y;
   const bool is_q = blockIdx.z == 0;
   const T* src = is_q ? q : k;
@@ -122,117 +130,120 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   const int nvalid = min(128, N - r0);
 
   // coalesced 16-byte loads of the valid rows
-  constexpr int VPR = D / 8;  // uint4 per row
   const uint4* g = reinterpret_cast<const uint4*>(src + ((size_t)bh * ldh + r0) * D);
-  uint4* s = reinterpret_cast<uint4*>(&tile[0][0]);
-  for (int i = threadIdx.x; i < nvalid * VPR; i += 256) s[i] = __ldg(g + i);
+  for (int i = threadIdx.x; i < nvalid * CPR; i += 256) {
+    const int r = i / CPR, j = i % CPR;
+    *reinterpret_cast<uint4*>(tile + RS * r + (j < CPH ? 16 * j : HO + 16 * (j - CPH))) = __ldg(g + i);
+  }
 
   if (is_q) {
     __syncthreads();
     if (threadIdx.x < D) {
       const int c = threadIdx.x;
+      const int off = c < D / 2 ? 2 * c : HO + 2 * (c - D / 2);
       float acc = 0.f;
-      for (int r = 0; r < nvalid; ++r) acc = __fadd_rn(acc, to_f32(tile[r][c]));
+      for (int r = 0; r < nvalid; ++r)
+        acc = __fadd_rn(acc, to_f32(*reinterpret_cast<const T*>(tile + RS * r + off)));
       const float m = __fdiv_rn(acc, (float)nvalid);
-      mean[c] = m;
+      mean[c < D / 2 ? c : MH + c - D / 2] = m;
       q_mean[((size_t)bh * NB + blk) * D + c] = m;
     }
   } else {
-    if (threadIdx.x < D) mean[threadIdx.x] = kmean[(size_t)bh * D + threadIdx.x];
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      mean[c < D / 2 ? c : MH + c - D / 2] = kmean[(size_t)bh * D + c];
+    }
   }
   __syncthreads();
 
   uint8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * D;
   float* scale = (is_q ? q_scale : k_scale) + (size_t)bh * Np + r0;
+  constexpr float kQmax = Q8 ? 127.f : 7.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = warp * 16 + (lane >> 1), hh = lane & 1;
+  const uint8_t* trow = tile + RS * r + HO * hh;
+  const float* mu = mean + MH * hh;
+  const bool valid = r < nvalid;
+  // eight smoothed values x - mean (fp32, RN) of chunk i of this lane's half
+  auto load8 = [&](int i, float (&x)[8]) {
+    unpack8<T>(*reinterpret_cast<const uint4*>(trow + 16 * i), x);
+    const float4 m0 = *reinterpret_cast<const float4*>(mu + 8 * i);
+    const float4 m1 = *reinterpret_cast<const float4*>(mu + 8 * i + 4);
+    const float2 d0 = __fadd2_rn(make_float2(x[0], x[1]), make_float2(-m0.x, -m0.y));
+    const float2 d1 = __fadd2_rn(make_float2(x[2], x[3]), make_float2(-m0.z, -m0.w));
+    const float2 d2 = __fadd2_rn(make_float2(x[4], x[5]), make_float2(-m1.x, -m1.y));
+    const float2 d3 = __fadd2_rn(make_float2(x[6], x[7]), make_float2(-m1.z, -m1.w));
+    x[0] = d0.x; x[1] = d0.y; x[2] = d1.x; x[3] = d1.y;
+    x[4] = d2.x; x[5] = d2.y; x[6] = d3.x; x[7] = d3.y;
+  };
+  // Pass 1: the row's amax (rows >= N are all zero)
+  float amax = 0.f;
+  if (valid) {
+#pragma unroll
+    for (int i = 0; i < CPH; ++i) {
+      float x[8];
+      load8(i, x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(x[u]));
+    }
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  const bool nz = amax > 0.f;                           // the scale may underflow to 0
+  const float sc = nz ? __fdiv_rn(amax, kQmax) : 0.f;
+  const float inv = nz ? __fdiv_rn(kQmax, amax) : 0.f;
+  const float2 inv2 = make_float2(inv, inv);
   // K^ rows are stored permuted inside each 128-row block: token j of the block
   // goes to stored row 8*((j/2) % 16) + 2*(j/32) + j % 2, so that stored row n
   // holds token 32*((n/2) % 4) + 2*(n/8) + n % 2 (the attention kernel's
   // .16x256b TMEM loads then give each thread 32 consecutive keys).  Q^ rows
   // keep their natural order.
-  constexpr int CPL = D / 32;  // channels per lane: 4 (D=128) or 2 (D=64)
-  constexpr float kQmax = Q8 ? 127.f : 7.f;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float mu[CPL];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) mu[i] = mean[lane * CPL + i];
-  // this lane's CPL consecutive channels of row r, smoothed (one 4- or 8-byte load)
-  auto load_row = [&](int r, float (&x)[CPL]) {
-    float raw[CPL];
-    if (CPL == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(&tile[r][lane * 4]);
-      const T* h = reinterpret_cast<const T*>(&u);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) raw[i] = to_f32(h[i]);
-    } else {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(&tile[r][lane * 2]);
-      const T* h = reinterpret_cast<const T*>(&u);
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) raw[i] = to_f32(h[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) x[i] = (r < nvalid) ? __fsub_rn(raw[i], mu[i]) : 0.f;
-  };
-  // The warp owns rows warp + 8j, j = 0..15.  Pass 1: every row's amax; lane j
-  // keeps row j's, so that the two IEEE divisions of all 16 rows take one
-  // instruction sequence of the warp instead of sixteen.
-  float my_amax = 0.f;
-#pragma unroll 4
-  for (int j = 0; j < 16; ++j) {
-    float x[CPL];
-    load_row(warp + 8 * j, x);
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) amax = fmaxf(amax, fabsf(x[i]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    my_amax = lane == j ? amax : my_amax;
-  }
-  const bool nz = my_amax > 0.f;
-  const float my_sc = nz ? __fdiv_rn(my_amax, kQmax) : 0.f;
-  const float my_inv = nz ? __fdiv_rn(kQmax, my_amax) : 0.f;
-  // Pass 2: quantize with row j's inverse scale (from lane j).
+  const int srow = is_q ? r : 8 * ((r >> 1) & 15) + 2 * (r >> 5) + (r & 1);
+  uint8_t* orow = out + (size_t)srow * D + (D / 2) * hh;
+  // Pass 2: quantize.  |x| <= amax and inv = RN(qmax/amax), so |x*inv| <=
+  // qmax*(1+2^-24)^2 < qmax + 1/2: the rounded value never leaves [-qmax,
+  // qmax] and needs no clamp.  Adding +0 turns a rounded -0 into +0 (the
+  // oracle's integer 0).
   // INT4 (the method): each value in [-7, 7] is stored as its e4m3 code:
   // every such integer is exact in e4m3, so the FP8 tensor path multiplies
   // the INT4 values exactly (at the same rate as the 8-bit integer path) and
   // yields S as an fp32 integer.  Zero is stored as +0 (code 0x00).
   // INT8 (the variant): values in [-127, 127] as two's-complement bytes.
-#pragma unroll 4
-  for (int j = 0; j < 16; ++j) {
-    const int r = warp + 8 * j;
-    const float inv = __shfl_sync(0xffffffffu, my_inv, j);
-    const float sc = __shfl_sync(0xffffffffu, my_sc, j);
-    const bool row_nz = __shfl_sync(0xffffffffu, my_amax, j) > 0.f;   // sc may underflow to 0
-    float x[CPL];
-    load_row(r, x);
-    uint32_t packed = 0;
-    if (row_nz) {
-      // |x| <= amax and inv = RN(qmax/amax), so |x*inv| <= qmax*(1+2^-24)^2 <
-      // qmax + 1/2: the rounded value never leaves [-qmax, qmax] and needs no
-      // clamp.  Adding +0 turns a rounded -0 into +0 (the oracle's integer 0).
-      float v[CPL];
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) v[i] = __fadd_rn(rintf(__fmul_rn(x[i], inv)), 0.f);
-      if (Q8) {
+  for (int i = 0; i < CPH; i += 2) {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (nz) {
 #pragma unroll
-        for (int i = 0; i < CPL; ++i)
-          packed |= (static_cast<uint32_t>(static_cast<int>(v[i])) & 0xFFu) << (8 * i);
-      } else {
-        // exact e4m3 codes of the integers, two per conversion
+      for (int c2 = 0; c2 < 2; ++c2) {
+        float x[8];
+        load8(i + c2, x);
+        float v[8];
 #pragma unroll
-        for (int i = 0; i < CPL; i += 2)
-          packed |= static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(v[i], v[i + 1]),
-                                                                     __NV_SATFINITE, __NV_E4M3))
-                    << (8 * i);
+        for (int u = 0; u < 8; u += 2) {
+          const float2 p = __fmul2_rn(make_float2(x[u], x[u + 1]), inv2);
+          v[u] = __fadd_rn(rintf(p.x), 0.f);
+          v[u + 1] = __fadd_rn(rintf(p.y), 0.f);
+        }
+#pragma unroll
+        for (int h4 = 0; h4 < 2; ++h4) {
+          uint32_t packed = 0;
+          if (Q8) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              packed |= (static_cast<uint32_t>(static_cast<int>(v[4 * h4 + u])) & 0xFFu) << (8 * u);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; u += 2)
+              packed |= static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+                            make_float2(v[4 * h4 + u], v[4 * h4 + u + 1]), __NV_SATFINITE, __NV_E4M3))
+                        << (8 * u);
+          }
+          w[2 * c2 + h4] = packed;
+        }
       }
     }
-    const int srow = is_q ? r : 8 * ((r >> 1) & 15) + 2 * (r >> 5) + (r & 1);
-    if (CPL == 4) {
-      reinterpret_cast<uint32_t*>(out + (size_t)srow * D)[lane] = packed;
-    } else {
-      reinterpret_cast<uint16_t*>(out + (size_t)srow * D)[lane] = static_cast<uint16_t>(packed);
-    }
-    if (lane == 0) scale[r] = sc;
+    *reinterpret_cast<uint4*>(orow + 8 * i) = make_uint4(w[0], w[1], w[2], w[3]);
   }
+  if (hh == 0) scale[r] = sc;
 }
 
 // ---------------------------------------------------------------------------
