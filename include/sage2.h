@@ -191,6 +191,9 @@ sage2_status sage2_attn_fwd_ex(const void* q, const void* k, const void* v, void
  *     (cudaGetSymbolAddress) and caches it: make it before any stream capture.
  *   - All calls share the array; each clears what must start at zero.  Calls
  *     whose GPU work overlaps race on it: order them on one stream.
+ *   - The cached address belongs to the device's context: after a
+ *     cudaDeviceReset of that device it is stale, and the library (this entry
+ *     and its memory pools alike) must not be called on that device again.
  * Arguments, layouts and other statuses as sage2_attn_fwd.
  */
 sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int B,

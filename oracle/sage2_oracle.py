@@ -65,12 +65,17 @@ INT8_MAX = 127      # symmetric INT8 range [-127, 127] (the INT8 variant)
 E4M3_MAX = 448.0    # largest finite e4m3 value; also the fixed P~ scale
 LOG2E = 1.4426950408889634
 
-# Relative distance from an e4m3 rounding boundary inside which the rounding of
-# 448*p is treated as ambiguous: the kernel evaluates p = exp2(x - m) in fp32
-# (x built from fp32 products and sums, exp2 with ~2 ulp error), so 448*p can
-# differ from the fp64 value by up to a few 1e-5 relative; either neighbouring
-# code is then a correct result.
-AMBIG_REL = 2.0 ** -13
+# Several correct results.  The decision that turns p into a code, e4m3(448 p),
+# is taken by the kernel in fp32: x' = sq*(sk*S) + C with C itself an fp32 dot
+# product, the running maximum of x', the argument x'*L - m*L + log2(448) and a
+# hardware exp2 approximation.  Where 448 p lies closer to an e4m3 rounding
+# boundary than the kernel's fp32 error can reach, either neighbouring code is
+# a correct result.  p448_band() bounds that error element by element; the
+# constants are the fp32 unit roundoff and the exp2 approximation's relative
+# error bound (ex2.approx.f32 is specified to a few ulp; 2^-21 covers 8 ulp).
+U32 = 2.0 ** -24
+EX2_REL = 2.0 ** -21
+LOG2_448 = math.log2(448.0)
 
 
 def n_pad(N: int) -> int:
@@ -136,13 +141,37 @@ def e4m3_round(x) -> np.ndarray:
     return e4m3_decode(e4m3_encode(x))
 
 
-def e4m3_ambiguity(y) -> np.ndarray:
-    """For y >= 0: |gap| between the two e4m3 neighbours if y lies within
-    AMBIG_REL (relative) of a rounding boundary, else 0."""
+def e4m3_neighbours(y, rel):
+    """For y >= 0 and a relative error bound rel (array or scalar): the e4m3
+    values that y*(1-rel) and y*(1+rel) round to.  They differ exactly where
+    an error of that size can move y across a rounding boundary."""
     y = np.asarray(y, np.float64)
-    lo = e4m3_round(y * (1.0 - AMBIG_REL))
-    hi = e4m3_round(y * (1.0 + AMBIG_REL))
-    return np.abs(hi - lo)
+    return e4m3_round(y * (1.0 - rel)), e4m3_round(y * (1.0 + rel))
+
+
+def p448_band(A, X, M, e_m, c_bound, L):
+    """Relative bound on how far the kernel's fp32 value of 448*p can be from
+    the exact 448*exp2(L*(X - M)), element by element.
+
+    A = sq_i*sk_j*S_ij and X = A + C_j (the unscaled score) in fp64; M the
+    exact running row maximum of X; c_bound the bound on the kernel's fp32
+    error in C_j; e_m the bound on the error of the kernel's running maximum
+    (the largest score error among the keys the row has seen).  With u the
+    fp32 unit roundoff, the kernel's score carries |x' - X| <= u(2|A| + |X|) +
+    c_bound (one rounding of sk*S, one of the fused multiply-add); its
+    argument x'L - mL + log2 448 adds the error of the maximum, the fp32
+    rounding of L (two roundings), and three roundings of values of the size
+    of L|X|, L|M|, the argument and log2 448.  exp2 turns an argument error
+    e into a relative error 2^e - 1 <= ln2 e (1 + e); its hardware
+    approximation adds EX2_REL.  The result is widened by 2^-20 for the
+    neglected second-order terms."""
+    e_x = U32 * (2.0 * np.abs(A) + np.abs(X)) + c_bound
+    arg = L * (X - M[:, None]) + LOG2_448
+    nb = LOG2_448 - L * M
+    darg = (L * (e_x + e_m[:, None])
+            + 2.0 * U32 * L * (np.abs(X) + 2.0 * np.abs(M)[:, None])
+            + U32 * (np.abs(nb)[:, None] + np.abs(arg) + 9.0))
+    return (math.log(2.0) * darg * (1.0 + darg) + EX2_REL) * (1.0 + 2.0 ** -20)
 
 
 # ----------------------------------------------------------------------------
@@ -268,6 +297,16 @@ def qk_correction(q_mean: np.ndarray, K: np.ndarray) -> np.ndarray:
     return C
 
 
+def qk_correction_bound(q_mean: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """The worst-case rounding error of C computed as an fp32 dot product of d
+    terms: d * u * sum_c |qbar_c K_jc| (u = 2^-24), shape as qk_correction."""
+    K = np.asarray(K, np.float64)
+    N, d = K.shape
+    Cb = np.zeros((q_mean.shape[0], n_pad(N)), np.float64)
+    Cb[:, :N] = d * U32 * (np.abs(np.asarray(q_mean, np.float64)) @ np.abs(K).T)
+    return Cb
+
+
 # ----------------------------------------------------------------------------
 # Step 5 - V to FP8 e4m3, one scale per channel over all tokens.
 # Reading: sv = amax/448, inv = 448/amax (float32 IEEE), code = e4m3(V*inv)
@@ -318,14 +357,19 @@ def qk_int(q_i4: np.ndarray, k_i4: np.ndarray) -> np.ndarray:
 
 
 def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
-                   q_blocks=None, quantize: bool = True):
+                   q_blocks=None, quantize: bool = True, explain_rows=None):
     """Online-softmax attention of one head over its payloads.
 
     p: dict with q_i4, q_scale, k_i4, k_scale, C (qk_correction), v_t, v_scale
-       (with quantize=False: 'q_s' / 'k_s' float rows replace q_i4*q_scale /
-       k_i4*k_scale and 'v' [N, d] replaces the e4m3 V; P~ is not rounded).
+       and optionally C_bound (the bound on the kernel's fp32 error in C, same
+       shape as C; 0 when absent) and v_mean (V smoothing).  With
+       quantize=False: 'q_s' / 'k_s' float rows replace q_i4*q_scale /
+       k_i4*k_scale and 'v' [N, d] replaces the e4m3 V; P~ is not rounded.
     q_blocks: iterable of 128-row query block indices to compute (default all).
-    Returns (O [rows, d] float64, amb [rows, d] float64, rows index array).
+    Returns (O [rows, d] float64, amb [rows, d] float64, rows index array);
+    with explain_rows (a collection of row indices) also a dict row ->
+    array [k, d]: the change of that output row that each of its k ambiguous
+    P~ codes would make if it were rounded to its other neighbour.
 
     Per query block and for key tiles in ascending order (causal: tiles above
     the diagonal skipped; masked scores are -inf), with L = sm_scale*log2(e):
@@ -336,8 +380,10 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
         inner= P~ . V~  over this tile only              (inner level)
         acc  = alpha*acc + inner                          (outer level)
     then O = acc * sv / (448 l), plus p['v_mean'] when V was smoothed.
-    'amb' bounds what a different but equally correct rounding of ambiguous
-    448p values (see AMBIG_REL) can change.
+    A code is ambiguous when the kernel's fp32 error bound (p448_band) can
+    move 448p across a rounding boundary; 'amb' is the sum of what all of a
+    row's ambiguous codes could change (a diagnostic: the parity tests ask
+    for the flips that explain a difference, one by one).
     """
     Np = n_pad(N)
     nb = Np // BM
@@ -356,10 +402,12 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
         vdec = np.zeros((Np, p["v"].shape[1])); vdec[:N] = p["v"]
         sv = np.ones(vdec.shape[1])
     C = np.asarray(p["C"], np.float64)
+    cbound = np.asarray(p["C_bound"], np.float64) if p.get("C_bound") is not None else np.zeros_like(C)
     d = vdec.shape[1]
     vbar = np.asarray(p["v_mean"], np.float64) if p.get("v_mean") is not None else np.zeros(d)
     blocks = range(nb) if q_blocks is None else q_blocks
-    outs, ambs, rows = [], [], []
+    want = set(int(i) for i in explain_rows) if explain_rows is not None else set()
+    outs, ambs, rows, expl = [], [], [], {}
     for b in blocks:
         r = np.arange(b * BM, min((b + 1) * BM, N))
         if r.size == 0:
@@ -368,11 +416,15 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
         l = np.zeros(r.size)
         acc = np.zeros((r.size, d))
         amb = np.zeros((r.size, d))
+        e_m = np.zeros(r.size)
+        track = [k for k, i in enumerate(r) if int(i) in want]
+        flips = {k: [] for k in track}                # per tracked row: flip vectors (acc units)
         last = b if causal else nb - 1
         for t in range(last + 1):
             c = np.arange(t * BN, (t + 1) * BN)
             S = qv[r] @ kv[c].T                                   # exact
-            x = (sq[r, None] * sk[None, c] * S + C[b][c][None, :]) * L
+            A = sq[r, None] * sk[None, c] * S
+            x = (A + C[b][c][None, :]) * L
             mask = c[None, :] >= N
             if causal:
                 mask = mask | (c[None, :] > r[:, None])
@@ -383,20 +435,38 @@ def attn_quantized(p: dict, N: int, causal: bool, sm_scale: float,
             l = alpha * l + pt.sum(axis=1)
             if quantize:
                 ph = e4m3_round(E4M3_MAX * pt)
-                gap = e4m3_ambiguity(E4M3_MAX * pt)
+                # the kernel's fp32 error bound, element by element
+                X = np.where(mask, 0.0, x / L)
+                cb = np.where(mask, 0.0, cbound[b][c][None, :])
+                e_m = np.maximum(e_m, np.max(U32 * (2.0 * np.abs(A) + np.abs(X)) + cb, axis=1))
+                rel = p448_band(np.where(mask, 0.0, A), X, m_new / L, e_m, cb, L)
+                lo, hi = e4m3_neighbours(E4M3_MAX * pt, rel)
+                gap = hi - lo
             else:
                 ph, gap = pt, np.zeros_like(pt)
             inner = ph @ vdec[c]                                  # inner level
             acc = alpha[:, None] * acc + inner                    # outer level
             amb = alpha[:, None] * amb + gap @ np.abs(vdec[c])
+            for k in track:
+                flips[k] = [f * alpha[k] for f in flips[k]]
+                for j in np.nonzero(gap[k] > 0)[0]:
+                    other = hi[k, j] if ph[k, j] == lo[k, j] else lo[k, j]
+                    flips[k].append((other - ph[k, j]) * vdec[c[j]])
             m = m_new
         scale = E4M3_MAX if quantize else 1.0
         outs.append(acc * sv[None, :] / (scale * l[:, None]) + vbar[None, :])
         ambs.append(amb * sv[None, :] / (scale * l[:, None]))
         rows.append(r)
+        for k in track:
+            f = np.array(flips[k]).reshape(-1, d)
+            expl[int(r[k])] = f * sv[None, :] / (scale * l[k])
     if not outs:
-        return np.zeros((0, d)), np.zeros((0, d)), np.zeros(0, np.int64)
-    return np.concatenate(outs), np.concatenate(ambs), np.concatenate(rows)
+        O, amb, rows = np.zeros((0, d)), np.zeros((0, d)), np.zeros(0, np.int64)
+    else:
+        O, amb, rows = np.concatenate(outs), np.concatenate(ambs), np.concatenate(rows)
+    if explain_rows is not None:
+        return O, amb, rows, expl
+    return O, amb, rows
 
 
 # ----------------------------------------------------------------------------
@@ -435,12 +505,23 @@ def sage2_head(Q, K, V, causal: bool, sm_scale: float | None = None, q_blocks=No
         sm_scale = 1.0 / math.sqrt(d)
     pay = smooth_quant_qk(Q, K, qk_bits)
     pay["C"] = qk_correction(pay["q_mean"], K)
+    pay["C_bound"] = qk_correction_bound(pay["q_mean"], K)
     if smooth_v:
         pay["v_t"], pay["v_scale"], pay["v_mean"] = quant_v_smoothed(V)
     else:
         pay["v_t"], pay["v_scale"] = quant_v(V)
     O, amb, rows = attn_quantized(pay, N, causal, sm_scale, q_blocks=q_blocks)
     return pay, O, amb, rows
+
+
+def flips_of_rows(pay: dict, N: int, causal: bool, sm_scale: float, rows) -> dict:
+    """For the given output rows of a head whose payloads are `pay` (as
+    sage2_head returns them): row -> [k, d] array, the change of the row that
+    each of its k ambiguous P~ codes makes when rounded to its other
+    neighbour (see attn_quantized)."""
+    rows = [int(i) for i in rows]
+    blocks = sorted({i // BM for i in rows})
+    return attn_quantized(pay, N, causal, sm_scale, q_blocks=blocks, explain_rows=rows)[3]
 
 
 # ----------------------------------------------------------------------------
@@ -452,9 +533,10 @@ def sage2_head(Q, K, V, causal: bool, sm_scale: float | None = None, q_blocks=No
 # ----------------------------------------------------------------------------
 
 def sage2_varlen_head(Q, K, V, cu_seqlens, causal: bool, sm_scale: float | None = None,
-                      qk_bits: int = 4, smooth_v: bool = False):
+                      qk_bits: int = 4, smooth_v: bool = False, with_payloads: bool = False):
     """One head of packed sequences: Q, K, V [T, d]; cu_seqlens [S+1] offsets.
-    Returns (O [T, d] float64, amb [T, d] float64)."""
+    Returns (O [T, d] float64, amb [T, d] float64); with_payloads also returns
+    the list of (first token, length, payload dict) of the non-empty sequences."""
     Q = np.asarray(Q, np.float32)
     T, d = Q.shape
     cu = [int(c) for c in cu_seqlens]
@@ -464,12 +546,15 @@ def sage2_varlen_head(Q, K, V, cu_seqlens, causal: bool, sm_scale: float | None 
         sm_scale = 1.0 / math.sqrt(d)
     O = np.zeros((T, d))
     amb = np.zeros((T, d))
+    pays = []
     for a, b in zip(cu, cu[1:]):
         if b == a:
             continue
-        _, o, m, rows = sage2_head(Q[a:b], K[a:b], V[a:b], causal, sm_scale,
-                                   qk_bits=qk_bits, smooth_v=smooth_v)
+        pay, o, m, rows = sage2_head(Q[a:b], K[a:b], V[a:b], causal, sm_scale,
+                                     qk_bits=qk_bits, smooth_v=smooth_v)
         O[a + rows] = o
         amb[a + rows] = m
+        pays.append((a, b - a, pay))
+    if with_payloads:
+        return O, amb, pays
     return O, amb
-

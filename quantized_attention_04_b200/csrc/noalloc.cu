@@ -19,7 +19,9 @@
 //    before anything is launched.
 //  - The first call on a device looks the array's device address up
 //    (cudaGetSymbolAddress, with that device current) and caches it; make that
-//    first call before any stream capture on that device.
+//    first call before any stream capture on that device.  The cached address
+//    belongs to the device's context: after a cudaDeviceReset of the device it
+//    is stale, so the library is not to be called on that device again.
 //  - Every call uses the same array and it keeps the previous call's
 //    contents.  What must start at zero (the per-channel |V| maximum) is
 //    cleared on the stream by every call; everything else is overwritten

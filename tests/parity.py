@@ -5,10 +5,15 @@ Tolerances (written here, used by every test):
   * payloads (INT4 values, e4m3 codes, every scale and mean): bit-exact;
   * the correction qk_corr (fp32 on the GPU, fp64 in the oracle): the fp32
     rounding bound of a d-term dot product, d * 2^-24 * sum_c |qbar_c K_c|;
-  * O: max-abs <= 2e-3 and relative L1 <= 1e-3 against the quantized oracle,
-    after removing the oracle's per-element ambiguity bound (elements whose
-    448*p sits within AMBIG_REL of an e4m3 rounding boundary may round either
-    way), plus half an ulp of the output dtype for fp16/bf16 outputs.
+  * O: relative L1 <= 1e-3 against the quantized oracle, on the raw
+    difference (only the output type's own rounding, half an ulp for
+    fp16/bf16 outputs, is taken off each element); and max-abs <= 2e-3 per
+    element, where a row that exceeds it passes only if rounding some of its
+    ambiguous P~ codes to their other neighbour (codes whose 448p lies within
+    the kernel's fp32 error bound of an e4m3 rounding boundary, see
+    oracle.p448_band) brings every element of the row within 2e-3.  The
+    flips are chosen one at a time from the oracle's list for that row; the
+    number used is reported.
 """
 from __future__ import annotations
 
@@ -43,19 +48,83 @@ def half_ulp(x: np.ndarray, dtype: torch.dtype) -> np.ndarray:
     return 0.5 * 2.0 ** (np.floor(np.log2(a)) - mant)
 
 
-def compare_o(got: np.ndarray, ref: np.ndarray, amb: np.ndarray, out_dtype) -> dict:
-    err = np.abs(got.astype(np.float64) - ref)
-    excess = np.maximum(err - amb - half_ulp(ref, out_dtype), 0.0)
-    stats = dict(max_abs=float(err.max()), max_excess=float(excess.max()),
+def explain_row(diff: np.ndarray, flips: np.ndarray, tol: np.ndarray):
+    """Greedy search for a set of flips (rows of `flips`, each used at most
+    once) whose sum brings every element of diff - sum within tol.  Returns
+    (explained, number of flips used)."""
+    res = diff.astype(np.float64).copy()
+    free = np.ones(len(flips), bool)
+
+    def cost(r):
+        return np.sum(np.maximum(np.abs(r) - tol, 0.0) ** 2, axis=-1)
+
+    cur = cost(res)
+    used = 0
+    while cur > 0:
+        if not free.any():
+            return False, used
+        cand = np.nonzero(free)[0]
+        costs = cost(res[None, :] - flips[cand])
+        k = int(np.argmin(costs))
+        if costs[k] >= cur:
+            return False, used
+        res = res - flips[cand[k]]
+        free[cand[k]] = False
+        cur = costs[k]
+        used += 1
+    return True, used
+
+
+def compare_o(got: np.ndarray, ref: np.ndarray, amb: np.ndarray, out_dtype, flips=None,
+              rows=None) -> dict:
+    """got, ref: [n, d].  flips: callable(list of row ids) -> {row id: [k, d]}
+    (the oracle's alternative roundings, oracle.flips_of_rows); rows: the row
+    id of each of the n rows (default 0..n-1)."""
+    got64 = got.astype(np.float64)
+    err = np.abs(got64 - ref)
+    ulp = half_ulp(np.maximum(np.abs(ref), np.abs(got64)), out_dtype)
+    excess = np.maximum(err - ulp, 0.0)
+    over_rows = np.nonzero((excess > MAX_ABS).any(axis=1))[0]
+    rows = np.arange(len(ref)) if rows is None else np.asarray(rows)
+    stats = dict(max_abs=float(err.max(initial=0.0)), max_excess=float(excess.max(initial=0.0)),
                  rel_l1=float(excess.sum() / max(np.abs(ref).sum(), 1e-30)),
-                 ambiguous=int((amb > 0).sum()))
+                 elems_over=int((excess > MAX_ABS).sum()), rows_over=int(len(over_rows)),
+                 flips_used=0, unexplained=[], amb_max=float(amb.max(initial=0.0)))
+    if len(over_rows):
+        table = flips([int(rows[i]) for i in over_rows]) if flips is not None else {}
+        for i in over_rows:
+            f = table.get(int(rows[i]), np.zeros((0, ref.shape[1])))
+            ok, n = explain_row(got64[i] - ref[i], f, MAX_ABS + ulp[i])
+            stats["flips_used"] += n
+            if not ok:
+                stats["unexplained"].append(int(rows[i]))
     return stats
 
 
-def assert_o_close(got, ref, amb, out_dtype, what=""):
-    s = compare_o(got, ref, amb, out_dtype)
-    assert s["max_excess"] <= MAX_ABS and s["rel_l1"] <= REL_L1, (what, s)
+def assert_o_close(got, ref, amb, out_dtype, what="", flips=None, rows=None):
+    s = compare_o(got, ref, amb, out_dtype, flips, rows)
+    assert s["rel_l1"] <= REL_L1 and not s["unexplained"], (what, s)
     return s
+
+
+def head_flips(pay, N, causal, sm_scale):
+    """The flips callable of compare_o for one head of the oracle."""
+    return lambda rows: orc.flips_of_rows(pay, N, causal, sm_scale, rows)
+
+
+def varlen_flips(pays, causal, sm_scale):
+    """The flips callable for one head of packed sequences: pays is the list
+    of (first token, length, payload) that oracle.sage2_varlen_head returns;
+    row ids are packed token indices."""
+    def flips(rows):
+        out = {}
+        for a, n, pay in pays:
+            mine = [r - a for r in rows if a <= r < a + n]
+            if mine:
+                for r, f in orc.flips_of_rows(pay, n, causal, sm_scale, mine).items():
+                    out[r + a] = f
+        return out
+    return flips
 
 
 def cosine(a: np.ndarray, b: np.ndarray) -> float:

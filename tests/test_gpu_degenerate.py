@@ -105,7 +105,8 @@ def test_degenerate_attention(qa, name, kw, causal):
     o = P.np32(o)
     assert np.isfinite(o).all()
     for h in range(q.shape[1]):
-        _, O, amb, rows = P.oracle_head(q, k, v, 0, h, causal, sm, smooth_v=smooth)
-        P.assert_o_close(o[0, h][rows], O, amb, torch.float32, (name, causal, h))
+        pay, O, amb, rows = P.oracle_head(q, k, v, 0, h, causal, sm, smooth_v=smooth)
+        P.assert_o_close(o[0, h][rows], O, amb, torch.float32, (name, causal, h),
+                         flips=P.head_flips(pay, q.shape[2], causal, sm), rows=rows)
     if name == "zero_all":
         assert (o == 0).all()

@@ -33,5 +33,6 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     o = P.np32(qa.sage2_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=cfg.causal, sm_scale=sm,
                                  out_dtype=torch.float32))
     assert qa.sage2_check_device_error() == 0
-    _, O, amb, rows = P.oracle_head(q, k, v, 0, 0, cfg.causal, sm)
-    P.assert_o_close(o[0, 0][rows], O, amb, torch.float32, "after timeout")
+    pay, O, amb, rows = P.oracle_head(q, k, v, 0, 0, cfg.causal, sm)
+    P.assert_o_close(o[0, 0][rows], O, amb, torch.float32, "after timeout",
+                     flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)

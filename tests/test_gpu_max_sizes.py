@@ -37,13 +37,15 @@ def _check(qa, q, k, v, causal, heads, blocks, out_dtype):
     assert qa.sage2_check_device_error() == 0
     for b, h in heads:
         opay, O, amb, rows = P.oracle_head(q, k, v, b, h, causal, sm, q_blocks=blocks)
-        opay["k_i4"] = opay["k_i4"][P.key_interleave(opay["k_i4"].shape[0])]
-        opay["q_i4"], opay["k_i4"] = P.int4_codes(opay["q_i4"]), P.int4_codes(opay["k_i4"])
+        lib = dict(opay)
+        lib["k_i4"] = lib["k_i4"][P.key_interleave(lib["k_i4"].shape[0])]
+        lib["q_i4"], lib["k_i4"] = P.int4_codes(lib["q_i4"]), P.int4_codes(lib["k_i4"])
         for n in ("q_i4", "q_scale", "k_i4", "k_scale", "k_mean"):
-            assert P.bits_equal(pay[n][b, h].cpu().numpy(), opay[n]), (n, b, h)
+            assert P.bits_equal(pay[n][b, h].cpu().numpy(), lib[n]), (n, b, h)
         got = P.np32(o[b, h])[rows]
         assert np.isfinite(got).all()
-        P.assert_o_close(got, O, amb, out_dtype, (b, h))
+        P.assert_o_close(got, O, amb, out_dtype, (b, h),
+                         flips=P.head_flips(opay, N, causal, sm), rows=rows)
 
 
 def test_most_heads(qa):

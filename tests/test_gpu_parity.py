@@ -119,8 +119,9 @@ def test_attention_small_full(qa, cfg, out_dtype):
     o = P.np32(o)
     for b in range(cfg.B):
         for h in range(cfg.H):
-            _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
-            P.assert_o_close(o[b, h][rows], O, amb, od, (cfg.name, b, h))
+            pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
+            P.assert_o_close(o[b, h][rows], O, amb, od, (cfg.name, b, h),
+                             flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
 
 
 def test_attention_quantized_entry_matches_full(qa):
@@ -145,19 +146,24 @@ def test_attention_config_full(qa, name):
     assert qa.sage2_check_device_error() == 0
     for b in range(cfg.B):
         for h in range(cfg.H):
-            _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
-            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (name, b, h))
+            pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
+            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (name, b, h),
+                             flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
 
 
+@pytest.mark.parametrize("out_dtype", ["input", torch.float32])
 @pytest.mark.parametrize("name", ["C3", "C4", "C5"])
-def test_attention_config_sampled(qa, name):
-    """Full-size launch (as the bench runs it: input-dtype output); sampled
-    heads and query blocks (first, middle, last -> diagonal and ragged tails)
-    compared with the oracle; payloads of the sampled heads bit-exact."""
+def test_attention_config_sampled(qa, name, out_dtype):
+    """Full-size launch (the bench's launch configuration; output in the input
+    dtype as the bench runs it, and in fp32 where the 2e-3 bound applies with
+    no output rounding); sampled heads and query blocks (first, middle, last
+    -> diagonal and ragged tails) compared with the oracle; payloads of the
+    sampled heads bit-exact."""
     cfg = CONFIGS[name]
     q, k, v, qd, kd, vd = _cuda(cfg)
     sm = P.default_scale(cfg.d)
-    o = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm)
+    od = cfg.torch_dtype if out_dtype == "input" else out_dtype
+    o = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out_dtype=od)
     pay = qa.sage2_smooth_quant_qk(qd, kd)
     torch.cuda.synchronize()
     assert qa.sage2_check_device_error() == 0
@@ -166,12 +172,15 @@ def test_attention_config_sampled(qa, name):
     blocks = sorted({0, nb // 2, nb - 1})
     for b, h in heads:
         opay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, q_blocks=blocks)
-        opay["k_i4"] = opay["k_i4"][P.key_interleave(opay["k_i4"].shape[0])]
-        opay["q_i4"], opay["k_i4"] = P.int4_codes(opay["q_i4"]), P.int4_codes(opay["k_i4"])
+        lib = dict(opay)
+        lib["k_i4"] = lib["k_i4"][P.key_interleave(lib["k_i4"].shape[0])]
+        lib["q_i4"], lib["k_i4"] = P.int4_codes(lib["q_i4"]), P.int4_codes(lib["k_i4"])
         for n in ("q_i4", "q_scale", "k_i4", "k_scale", "k_mean"):
-            assert P.bits_equal(pay[n][b, h].cpu().numpy(), opay[n]), (name, n)
+            assert P.bits_equal(pay[n][b, h].cpu().numpy(), lib[n]), (name, n)
         got = P.np32(o[b, h])[rows]
-        P.assert_o_close(got, O, amb, cfg.torch_dtype, (name, b, h))
+        stats = P.assert_o_close(got, O, amb, od, (name, b, h),
+                                 flips=P.head_flips(opay, cfg.N, cfg.causal, sm), rows=rows)
+        print(name, od, (b, h), stats)
         ref = orc.attn_fp64(P.np32(q[b, h]), P.np32(k[b, h]), P.np32(v[b, h]), cfg.causal, sm,
                             rows=rows)
         assert abs(P.cosine(got, ref) - P.cosine(O, ref)) < 1e-4

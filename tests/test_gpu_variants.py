@@ -82,8 +82,9 @@ def test_int8_attention_small(qa, cfg):
     assert qa.sage2_check_device_error() == 0
     for b in range(cfg.B):
         for h in range(cfg.H):
-            _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, qk_bits=8)
-            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (cfg.name, b, h))
+            pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, qk_bits=8)
+            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (cfg.name, b, h),
+                             flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
 
 
 # ------------------------------------------------------------- V smoothing
@@ -112,9 +113,10 @@ def test_smoothed_v_attention_small(qa, cfg, qk_bits):
     assert qa.sage2_check_device_error() == 0
     for b in range(cfg.B):
         for h in range(cfg.H):
-            _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, qk_bits=qk_bits,
-                                            smooth_v=True)
-            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (cfg.name, qk_bits, b, h))
+            pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, qk_bits=qk_bits,
+                                              smooth_v=True)
+            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (cfg.name, qk_bits, b, h),
+                             flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
 
 
 def test_variant_stage_calls_match_full_call(qa):
@@ -145,7 +147,8 @@ def test_variants_config_sampled(qa, name):
         torch.cuda.synchronize()
         assert qa.sage2_check_device_error() == 0
         b, h = cfg.B - 1, cfg.H - 1
-        _, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, q_blocks=blocks,
-                                        qk_bits=qk_bits, smooth_v=smooth_v)
+        pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm, q_blocks=blocks,
+                                          qk_bits=qk_bits, smooth_v=smooth_v)
         P.assert_o_close(P.np32(o[b, h])[rows], O, amb, cfg.torch_dtype,
+                         flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows, what=
                          (name, qk_bits, smooth_v))

@@ -49,9 +49,11 @@ def test_varlen_matches_oracle(qa, cu, H, d, dtype, causal, qk_bits, smooth_v):
     assert qa.sage2_check_device_error() == 0
     o = P.np32(o)
     for h in range(H):
-        O, amb = orc.sage2_varlen_head(P.np32(q[h]), P.np32(k[h]), P.np32(v[h]), cu, causal, sm,
-                                       qk_bits=qk_bits, smooth_v=smooth_v)
-        P.assert_o_close(o[h], O, amb, torch.float32, (cu, h))
+        O, amb, pays = orc.sage2_varlen_head(P.np32(q[h]), P.np32(k[h]), P.np32(v[h]), cu,
+                                             causal, sm, qk_bits=qk_bits, smooth_v=smooth_v,
+                                             with_payloads=True)
+        P.assert_o_close(o[h], O, amb, torch.float32, (cu, h),
+                         flips=P.varlen_flips(pays, causal, sm))
 
 
 def test_varlen_equal_lengths_equal_batched_call(qa):

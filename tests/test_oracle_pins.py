@@ -79,11 +79,74 @@ def test_e4m3_encode_matches_torch_converter_random():
     assert same.all(), x[~same][:10]
 
 
-def test_e4m3_ambiguity_flags_only_near_boundaries():
-    # exactly representable -> never ambiguous; a midpoint -> ambiguous
-    assert orc.e4m3_ambiguity(np.array([1.0]))[0] == 0
-    assert orc.e4m3_ambiguity(np.array([1.0625]))[0] == pytest.approx(0.125)
-    assert orc.e4m3_ambiguity(np.array([1.0625 * (1 + 4 * orc.AMBIG_REL)]))[0] == 0
+def test_e4m3_neighbours_differ_only_near_boundaries():
+    # exactly representable -> one value; a boundary -> both neighbours
+    lo, hi = orc.e4m3_neighbours(np.array([1.0, 1.0625, 368.0, 368.0 * (1 + 2 ** -10)]), 2 ** -12)
+    assert lo[0] == hi[0] == 1.0
+    assert (lo[1], hi[1]) == (1.0, 1.125)
+    assert (lo[2], hi[2]) == (352.0, 384.0)
+    assert lo[3] == hi[3] == 384.0
+
+
+def _band_case(rng, n, d, cmag):
+    """Random scores of one row as the kernel forms them: exact integer S,
+    fp32 scales, a correction of magnitude cmag, and its error bound."""
+    S = rng.integers(-49 * d // 4, 49 * d // 4 + 1, n).astype(np.float64)
+    sq = np.float32(rng.uniform(0.05, 3.0))
+    sk = rng.uniform(0.05, 3.0, n).astype(np.float32)
+    C = (rng.standard_normal(n) * cmag).astype(np.float64)
+    cb = d * orc.U32 * np.abs(C) * rng.uniform(1.0, 4.0, n)
+    return S, sq, sk, C, cb
+
+
+def _f32(x):
+    return np.asarray(x, np.float64).astype(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_p448_band_covers_an_fp32_evaluation(seed):
+    """The band must contain what an fp32 evaluation of the kernel's formula
+    gives: sk*S and the fused multiply-add rounded to fp32, a correction
+    anywhere within its error bound, the running maximum taken over the fp32
+    scores, the argument x'L - mL + log2 448 in fp32 (L itself rounded), and
+    an exp2 off by up to EX2_REL."""
+    rng = np.random.default_rng(300 + seed)
+    d = 128
+    sm = 1.0 / math.sqrt(d) * rng.uniform(0.5, 4.0)
+    L = sm * orc.LOG2E
+    Lf = _f32(_f32(sm) * _f32(orc.LOG2E))
+    worst = 0.0
+    for _ in range(40):
+        S, sq, sk, C, cb = _band_case(rng, 256, d, rng.choice([0.1, 10.0, 1000.0]))
+        A = np.float64(sq) * sk.astype(np.float64) * S
+        X = A + C
+        M = np.array([X.max()])
+        e_m = np.array([np.max(orc.U32 * (2 * np.abs(A) + np.abs(X)) + cb)])
+        band_all = orc.p448_band(A[None], X[None], M, e_m, cb[None], L)[0]
+        y = 448.0 * np.exp2(L * (X - M[0]))
+        for trial in range(4):
+            Cf = _f32(C + cb * rng.uniform(-1, 1, C.size))
+            t = _f32(sk.astype(np.float64) * S)
+            xk = _f32(np.float64(sq) * t + Cf)
+            mk = xk.max()
+            nb = _f32(_f32(orc.LOG2_448) - _f32(mk * Lf))
+            arg = _f32(xk * Lf + nb)
+            yk = np.exp2(arg) * (1 + orc.EX2_REL * rng.uniform(-1, 1, arg.size))
+            live = y > 448.0 * 2.0 ** -40
+            rel = np.abs(yk[live] / y[live] - 1)
+            band = band_all[live]
+            assert (rel <= band).all(), (rel / band).max()
+            worst = max(worst, float((rel / band).max()))
+    assert worst > 0.01          # the band is not vacuously wide
+
+
+def test_p448_band_grows_with_each_error_source():
+    A = np.array([[100.0]]); X = np.array([[90.0]]); M = np.array([95.0]); L = 0.2
+    base = orc.p448_band(A, X, M, np.array([0.0]), np.array([[0.0]]), L)[0, 0]
+    assert orc.p448_band(A, X, M, np.array([1e-3]), np.array([[0.0]]), L)[0, 0] > base
+    assert orc.p448_band(A, X, M, np.array([0.0]), np.array([[1e-3]]), L)[0, 0] > base
+    assert orc.p448_band(A * 10, X, M, np.array([0.0]), np.array([[0.0]]), L)[0, 0] > base
+    assert base >= orc.EX2_REL
 
 
 # --------------------------------------------------------------------- INT4
@@ -193,6 +256,76 @@ def test_online_softmax_identity_quant_equals_fp64(N, causal):
     assert np.array_equal(rows, np.arange(N))
     assert np.abs(O - ref).max() < 1e-11
     assert (amb == 0).all()
+
+
+def _golden():
+    vals = {}
+    for line in open(os.path.join(GOLDEN, "two_tile_recurrence.txt")):
+        line = line.split("#")[0].strip()
+        if line:
+            key, val = line.split()
+            vals[key] = float(val)
+    return vals
+
+
+def scripted_payload(x_tile0, x_tile1, v0, v1, d=64):
+    """One head, N = 256, not causal: Q^ = K^ = 0 with unit scales, so the
+    score of key j (in log2 units, with sm_scale = 1) is the correction
+    alone; x_tile*: [128] scores; v0, v1: per-channel V values of each tile
+    (exact e4m3 values, v_scale 1).  The same scores for both query blocks."""
+    N = 256
+    x = np.concatenate([x_tile0, x_tile1])
+    vt = np.zeros((d, N), np.uint8)
+    vt[:, :128] = orc.e4m3_encode(np.asarray(v0, np.float64))[:, None]
+    vt[:, 128:] = orc.e4m3_encode(np.asarray(v1, np.float64))[:, None]
+    return dict(q_i4=np.zeros((N, d), np.int8), q_scale=np.ones(N, np.float32),
+                k_i4=np.zeros((N, d), np.int8), k_scale=np.ones(N, np.float32),
+                C=np.repeat((x / orc.LOG2E)[None, :], 2, axis=0), v_t=vt,
+                v_scale=np.ones(d, np.float32))
+
+
+def scenario_a(d=64):
+    x0 = np.r_[np.zeros(64), np.full(64, -0.3)]
+    x1 = np.r_[np.full(32, 0.7), np.full(96, 0.2)]
+    v1 = np.where(np.arange(d) % 2 == 0, 2.0, -0.5)
+    return scripted_payload(x0, x1, np.ones(d), v1, d)
+
+
+def scenario_b(d=64):
+    x0 = np.full(128, -30.0)
+    x0[0] = 0.0
+    x0[1] = math.log2(368.0 / 448.0) + math.log2(1 + 2.0 ** -22)
+    x1 = np.full(128, -30.0)
+    x1[0] = 0.5
+    v0 = np.where(np.arange(d) % 2 == 0, 1.0, -2.0)
+    return scripted_payload(x0, x1, v0, np.full(d, 0.5), d)
+
+
+def test_two_tile_recurrence_golden():
+    """Rounding P~ per tile against the running maximum, then rescaling by
+    alpha into the outer accumulator, against the hand-worked values."""
+    g = _golden()
+    O, amb, rows = orc.attn_quantized(scenario_a(), 256, False, 1.0)
+    assert np.array_equal(rows, np.arange(256))
+    assert np.allclose(O[:, 0::2], g["A_O_even"], rtol=1e-12, atol=0)
+    assert np.allclose(O[:, 1::2], g["A_O_odd"], rtol=1e-12, atol=0)
+    assert (amb == 0).all()                # no score near a boundary
+
+
+def test_ambiguous_code_and_its_flip_golden():
+    """One 448p sits 2^-22 above an e4m3 boundary: the oracle rounds it up,
+    lists it as its only ambiguous code, and gives the hand-worked change of
+    the output when it is rounded down instead."""
+    g = _golden()
+    O, amb, rows, flips = orc.attn_quantized(scenario_b(), 256, False, 1.0, explain_rows=[0, 200])
+    assert np.allclose(O[:, 0::2], g["B_O_even"], rtol=1e-12, atol=0)
+    assert np.allclose(O[:, 1::2], g["B_O_odd"], rtol=1e-12, atol=0)
+    for row in (0, 200):
+        f = flips[row]
+        assert f.shape == (1, 64)
+        assert np.allclose(f[0, 0::2], g["B_delta_even"], rtol=1e-12, atol=0)
+        assert np.allclose(f[0, 1::2], g["B_delta_odd"], rtol=1e-12, atol=0)
+    assert np.allclose(amb[0], np.abs(flips[0][0]), rtol=1e-12)
 
 
 @pytest.mark.parametrize("N", [1, 5, 100, 128])
