@@ -16,8 +16,9 @@ Under torchrun each rank runs its own full copy of the workload (heads are
 independent: no collective on the data path), so scaling is weak.  Rank 0
 prints one JSON line.
 
---impl reference times the CPU oracle (the plain numpy restatement of the
-method) on a bounded sample of the same workload, on the host cores.
+--impl reference times the CPU oracle (the plain C restatement of the method,
+oracle/sage2_oracle.c, OpenMP on every host core) on a bounded sample of the
+same workload; the cpu_baseline leg times the same sample.
 """
 from __future__ import annotations
 
@@ -50,17 +51,6 @@ def load_peaks():
         d = json.load(open(p))
         return d["bf16_tflops"], d.get("bf16_tflops_sustained"), d["hbm_gbs"], "measured"
     return 1590.0, 1400.0, 6650.0, "fallback"
-
-
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
 
 
 # ---------------------------------------------------------------- clocks
@@ -187,32 +177,40 @@ def recorded_traffic(workload: str):
 
 
 # ---------------------------------------------------------------- oracle leg
-def oracle_sample(cfg, q, k, v, n_blocks: int, qk_bits: int = 4, smooth_v: bool = False):
-    """Time the CPU oracle on head (0,0): its payloads plus n_blocks query
-    blocks spread over the sequence.  Returns (ops, seconds, description)."""
-    from oracle import sage2_oracle as orc
-    N, d = cfg.N, cfg.d
-    nb = (N + 127) // 128
-    blocks = sorted(set(int(x) for x in np.linspace(0, nb - 1, n_blocks)))
+REF_BLOCKS = 8   # query blocks of head (0,0) in one CPU sample
+
+
+def sample_blocks(cfg, n_blocks: int = REF_BLOCKS):
+    nb = (cfg.N + 127) // 128
+    return sorted(set(int(x) for x in np.linspace(0, nb - 1, n_blocks)))
+
+
+def oracle_sample(cfg, q, k, v, qk_bits: int = 4):
+    """One CPU sample: the plain C oracle (oracle/sage2_oracle.c) on head (0,0)
+    of the workload: the head's smoothing, INT4/INT8 and FP8 payloads, then
+    the correction and the quantized attention of REF_BLOCKS query blocks
+    spread over the sequence, the blocks in parallel on every host core
+    (OpenMP).  Returns (ops, seconds, description); ops counts 4 d per
+    (query, visible key) of the sampled rows, the metric's own unit."""
+    from oracle import c_oracle as corc
+    blocks = sample_blocks(cfg)
     Q = q[0, 0].float().numpy()
     K = k[0, 0].float().numpy()
     V = v[0, 0].float().numpy()
-    sm = 1.0 / math.sqrt(d)
+    sm = 1.0 / math.sqrt(cfg.d)
     t0 = time.perf_counter()
-    orc.sage2_head(Q, K, V, cfg.causal, sm, q_blocks=blocks, qk_bits=qk_bits, smooth_v=smooth_v)
+    _, ops = corc.sample_forward(Q, K, V, cfg.causal, sm, blocks, qk_bits)
     dt = time.perf_counter() - t0
-    ops = 0.0
-    for b in blocks:
-        rows = np.arange(b * 128, min((b + 1) * 128, N))
-        vis = (rows + 1) if cfg.causal else np.full(rows.size, N)
-        ops += 4.0 * d * float(vis.sum())
-    if cfg.causal:
-        # the metric counts half of the dense 4*N^2*d for causal; the exact
-        # visible-key count above is that half (up to the diagonal's N terms)
-        pass
-    desc = (f"head (0,0) of {cfg.name}: full smoothing/quantization of the head + "
-            f"{len(blocks)} of {nb} query blocks {blocks[:3]}..{blocks[-1:]}")
+    nb = (cfg.N + 127) // 128
+    desc = (f"plain C oracle, head (0,0) of {cfg.name}: smoothing/quantization of the whole "
+            f"head + correction and attention of {len(blocks)} of {nb} query blocks "
+            f"{blocks[:2]}..{blocks[-1:]} (OpenMP over blocks)")
     return ops, dt, desc
+
+
+def host_cores() -> int:
+    from oracle import c_oracle as corc
+    return corc.threads()
 
 
 def run_reference(args, cfg, world, rank):
@@ -222,13 +220,13 @@ def run_reference(args, cfg, world, rank):
     times, opss = [], []
     desc = ""
     for _ in range(args.warmup):
-        oracle_sample(cfg, q, k, v, 1, args.qk_bits, args.smooth_v)
+        oracle_sample(cfg, q, k, v, args.qk_bits)
     for _ in range(args.steps):
-        ops, dt, desc = oracle_sample(cfg, q, k, v, args.ref_blocks, args.qk_bits, args.smooth_v)
+        ops, dt, desc = oracle_sample(cfg, q, k, v, args.qk_bits)
         times.append(dt)
         opss.append(ops)
     value = sum(opss) / sum(times) / 1e12
-    cores = blas_threads()
+    cores = host_cores()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -259,9 +257,10 @@ def run_sage2(args, cfg, world, rank, local):
     od = torch.empty_like(qd)
     stream = torch.cuda.current_stream(dev)
 
-    variant = ("int4" if args.qk_bits == 4 else "int8") + ("+smooth_v" if args.smooth_v else "")
+    variant = ("int4" if args.qk_bits == 4 else "int8") + ("-packed" if args.packed else "") \
+        + ("+smooth_v" if args.smooth_v else "")
     # Payload buffers are allocated once, by the caller, as the C ABI allows.
-    pay = qa.sage2_smooth_quant_qk(qd, kd, qk_bits=args.qk_bits)
+    pay = qa.sage2_smooth_quant_qk(qd, kd, qk_bits=args.qk_bits, packed=args.packed)
     vpay = qa.sage2_quant_v(vd, smooth=args.smooth_v)
     # The timed step runs the three stage calls of the C ABI (the same kernels,
     # in the same order, as sage2_attn_fwd) so that the attention launch can be
@@ -269,7 +268,8 @@ def run_sage2(args, cfg, world, rank, local):
     attn_ev = []
 
     def step(record: bool):
-        qa.sage2_smooth_quant_qk(qd, kd, out=pay, qk_bits=args.qk_bits)
+        qa.sage2_smooth_quant_qk(qd, kd, out=pay, qk_bits=args.qk_bits, packed=args.packed,
+                                 causal_corr=cfg.causal)
         qa.sage2_quant_v(vd, out=vpay, smooth=args.smooth_v)
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -346,12 +346,19 @@ def run_sage2(args, cfg, world, rank, local):
                "h2d_bytes_per_step": int(3 * qh.numel() * qh.element_size()),
                "d2h_bytes_per_step": int(oh.numel() * oh.element_size())}
 
-    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    # ---- CPU oracle baseline (rank 0, N = 1 only): the reference arm's
+    # sample, repeated for about ten seconds of CPU work
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ops, dt, desc = oracle_sample(cfg, q, k, v, args.cpu_blocks, args.qk_bits, args.smooth_v)
-        cpu = {"value": ops / dt / 1e12, "unit": "TOPS", "cores": blas_threads(),
-               "kind": "oracle", "sample": desc, "seconds": dt}
+        tot_ops = tot_s = 0.0
+        reps = 0
+        while reps < 20 and (tot_s < 10.0 or reps < 2):
+            ops, dt, desc = oracle_sample(cfg, q, k, v, args.qk_bits)
+            tot_ops += ops
+            tot_s += dt
+            reps += 1
+        cpu = {"value": tot_ops / tot_s / 1e12, "unit": "TOPS", "cores": host_cores(),
+               "kind": "oracle", "sample": f"{desc}; {reps} samples", "seconds": tot_s}
 
     if rank == 0:
         line = {
@@ -466,7 +473,7 @@ def run_sweep(args, world, rank, local):
             attn_ev = []
 
             def step(record):
-                qa.sage2_smooth_quant_qk(qd, kd, out=pay)
+                qa.sage2_smooth_quant_qk(qd, kd, out=pay, causal_corr=True)
                 qa.sage2_quant_v(vd, out=vpay)
                 if record:
                     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -518,13 +525,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sage2", choices=["sage2", "reference"])
     ap.add_argument("--config", default="C5", choices=sorted(CONFIGS))
-    ap.add_argument("--ref-blocks", type=int, default=8,
-                    help="query blocks per step of the oracle in --impl reference")
-    ap.add_argument("--cpu-blocks", type=int, default=48,
-                    help="query blocks of the oracle sample behind cpu_baseline")
     ap.add_argument("--qk-bits", type=int, default=4, choices=[4, 8],
                     help="4: the method (INT4 Q/K); 8: the INT8 variant")
     ap.add_argument("--smooth-v", action="store_true", help="the V-smoothing variant")
+    ap.add_argument("--packed", action="store_true",
+                    help="INT4 payloads stored two per byte (expanded before the attention kernel)")
     ap.add_argument("--sweep", action="store_true",
                     help="the causal bf16 sweep d x N at B=1, H=32 (one line per point)")
     ap.add_argument("--varlen", type=int, default=0,

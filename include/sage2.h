@@ -79,8 +79,19 @@ typedef enum { SAGE2_F16 = 0, SAGE2_BF16 = 1, SAGE2_F32 = 2 } sage2_dtype;
  *                   research/19 summary).  Values in [-127,127] stored as
  *                   two's-complement bytes; scale = amax/127.  Everything else on
  *                   the path is unchanged (smoothing, correction, FP8 P~V).
+ *   SAGE2_QK_INT4_PACKED : the method's INT4 values (the same values and
+ *                   scales as SAGE2_QK_INT4) stored two per byte, the INT4
+ *                   storage precision of the abstract: q_i4 and k_i4 are
+ *                   [B,H,Np,d/2] bytes; byte c of a row holds channel 2c in
+ *                   bits 3:0 and channel 2c+1 in bits 7:4, each a
+ *                   two's-complement nibble; k_i4 rows are permuted as for
+ *                   SAGE2_QK_INT4.  B200 has no INT4 tensor-core path, so the
+ *                   attention entries expand the nibbles to e4m3 codes (one
+ *                   memory-bound pass into library scratch) before the
+ *                   attention kernel: the output is bit-identical to that of
+ *                   SAGE2_QK_INT4.  Not accepted by sage2_debug_qk_s32_ex.
  */
-typedef enum { SAGE2_QK_INT4 = 0, SAGE2_QK_INT8 = 1 } sage2_qk_format;
+typedef enum { SAGE2_QK_INT4 = 0, SAGE2_QK_INT8 = 1, SAGE2_QK_INT4_PACKED = 2 } sage2_qk_format;
 
 /*
  * Smoothing + INT4 quantization of Q and K, and the Q-smoothing correction.
@@ -102,7 +113,13 @@ sage2_status sage2_smooth_quant_qk(const void* q, const void* k, int dtype, int 
 
 /* As sage2_smooth_quant_qk with the payload format chosen by `qk_format`
  * (sage2_qk_format; SAGE2_ERR_INVALID_ARG otherwise).  INT8: scale = amax/127,
- * q = clamp(rint(x * (127/amax)), -127, 127) as int8 bytes. */
+ * q = clamp(rint(x * (127/amax)), -127, 127) as int8 bytes.
+ * qk_format may carry the flag SAGE2_QK_CAUSAL_CORR (OR-ed in): qk_corr is then
+ * written only where a causal attention reads it, i.e. qk_corr[blk][j] for key
+ * tiles j/128 <= blk, in whole 32-block groups (at least those entries are
+ * written; the others keep what the buffer held).  sage2_attn_fwd does the
+ * same for causal calls. */
+#define SAGE2_QK_CAUSAL_CORR 0x100
 sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, int B, int H, int N,
                                       int d, uint8_t* q_i4, float* q_scale, float* q_mean,
                                       uint8_t* k_i4, float* k_scale, float* k_mean,

@@ -25,8 +25,19 @@ __all__ = [
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage2.so")
 F16, BF16, F32 = 0, 1, 2
-QK_INT4, QK_INT8 = 0, 1
+QK_INT4, QK_INT8, QK_INT4_PACKED = 0, 1, 2
 _QKF = {4: QK_INT4, 8: QK_INT8}
+
+
+def _fmt(qk_bits: int, packed: bool = False) -> int:
+    """sage2_qk_format of (qk_bits, packed): packed is two INT4 values per byte."""
+    if qk_bits not in _QKF:
+        raise ValueError("qk_bits must be 4 or 8")
+    if packed:
+        if qk_bits != 4:
+            raise ValueError("packed storage is for INT4 values (qk_bits=4)")
+        return QK_INT4_PACKED
+    return _QKF[qk_bits]
 _DT = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
 STATUS = {0: "SAGE2_OK", 1: "SAGE2_ERR_INVALID_ARG", 2: "SAGE2_ERR_UNSUPPORTED",
           3: "SAGE2_ERR_MISALIGNED", 4: "SAGE2_ERR_CUDA", 5: "SAGE2_ERR_NO_MEM",
@@ -134,15 +145,29 @@ def _qk_bits_of(t: torch.Tensor) -> int:
     return 8 if t.dtype == torch.int8 else 4
 
 
+def _format_of(pay: dict) -> int:
+    """sage2_qk_format of a payload dict: int8 -> INT8; uint8 rows of d/2
+    bytes (d from q_mean) -> packed INT4; uint8 rows of d bytes -> INT4 codes."""
+    if pay["q_i4"].dtype == torch.int8:
+        return QK_INT8
+    return QK_INT4_PACKED if 2 * pay["q_i4"].shape[-1] == pay["q_mean"].shape[-1] else QK_INT4
+
+
+QK_CAUSAL_CORR = 0x100
+
+
 def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = None,
-                          qk_bits: int = 4) -> dict:
+                          qk_bits: int = 4, packed: bool = False,
+                          causal_corr: bool = False) -> dict:
     """Smoothing + INT4 (qk_bits=4, the method) or INT8 (qk_bits=8, the variant)
     of Q and K and the Q-smoothing correction.  Returns the payload dict (q_i4,
     q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr); q_i4/k_i4 are uint8 e4m3
-    codes for INT4 and int8 values for INT8.  `out`, if given, is such a dict
-    (from an earlier call with the same qk_bits) and is overwritten."""
-    if qk_bits not in _QKF:
-        raise ValueError("qk_bits must be 4 or 8")
+    codes for INT4, int8 values for INT8, and with packed=True (INT4 only)
+    uint8 [B,H,Np,d/2] bytes of two two's-complement nibbles (channel 2c in
+    bits 3:0).  `out`, if given, is such a dict (from an earlier call with the
+    same format) and is overwritten.  causal_corr writes qk_corr only where
+    a causal attention reads it (key tile <= query block)."""
+    fmt = _fmt(qk_bits, packed)
     B, H, N, d = _dims(q)
     if k.shape != q.shape or k.dtype != q.dtype:
         raise ValueError("q and k must have the same shape and dtype")
@@ -151,24 +176,25 @@ def sage2_smooth_quant_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = N
     NB = Np // 128
     dev = q.device
     if out is None:
-        out = _qk_payloads(B, H, Np, NB, d, dev, qk_bits)
-    elif _qk_bits_of(out["q_i4"]) != qk_bits:
-        raise ValueError("out holds payloads of the other qk_bits")
+        out = _qk_payloads(B, H, Np, NB, d, dev, qk_bits, packed)
+    elif _format_of(out) != fmt:
+        raise ValueError("out holds payloads of another format")
     st = lib().sage2_smooth_quant_qk_ex(
         _ptr(q), _ptr(k), _DT[q.dtype], B, H, N, d, _ptr(out["q_i4"]), _ptr(out["q_scale"]),
         _ptr(out["q_mean"]), _ptr(out["k_i4"]), _ptr(out["k_scale"]), _ptr(out["k_mean"]),
-        _ptr(out["qk_corr"]), _QKF[qk_bits], _stream(q))
+        _ptr(out["qk_corr"]), fmt | (QK_CAUSAL_CORR if causal_corr else 0), _stream(q))
     _check("sage2_smooth_quant_qk_ex", st)
     return out
 
 
-def _qk_payloads(B, H, Np, NB, d, dev, qk_bits=4) -> dict:
+def _qk_payloads(B, H, Np, NB, d, dev, qk_bits=4, packed=False) -> dict:
     ity = torch.uint8 if qk_bits == 4 else torch.int8   # e4m3 codes of INT4 values / INT8 values
+    w = d // 2 if packed else d                          # bytes per payload row
     return dict(
-        q_i4=torch.empty(B, H, Np, d, dtype=ity, device=dev),
+        q_i4=torch.empty(B, H, Np, w, dtype=ity, device=dev),
         q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
         q_mean=torch.empty(B, H, NB, d, dtype=torch.float32, device=dev),
-        k_i4=torch.empty(B, H, Np, d, dtype=ity, device=dev),   # rows permuted per block
+        k_i4=torch.empty(B, H, Np, w, dtype=ity, device=dev),   # rows permuted per block
         k_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
         k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev),
         qk_corr=torch.empty(B, H, NB, Np, dtype=torch.float32, device=dev),
@@ -199,16 +225,18 @@ def sage2_attn_fwd_quantized(pay: dict, v_fp8_t: torch.Tensor, v_scale: torch.Te
                              out: torch.Tensor | None = None,
                              v_mean: torch.Tensor | None = None) -> torch.Tensor:
     """The attention kernel alone, over payloads from sage2_smooth_quant_qk /
-    sage2_quant_v (or any tensors in those layouts).  The payload format (INT4 or
-    INT8) follows the q_i4 dtype; v_mean is the token mean of a smoothed V."""
-    B, H, Np, d = pay["q_i4"].shape
+    sage2_quant_v (or any tensors in those layouts).  The payload format (INT4
+    codes, packed INT4 or INT8) follows the q_i4 dtype and row width; v_mean
+    is the token mean of a smoothed V."""
+    B, H, Np = pay["q_i4"].shape[:3]
+    d = pay["q_mean"].shape[-1]
     if out is None:
         out = torch.empty(B, H, N, d, dtype=out_dtype, device=pay["q_i4"].device)
     st = lib().sage2_attn_fwd_quantized_ex(
         _ptr(pay["q_i4"]), _ptr(pay["q_scale"]), _ptr(pay["k_i4"]), _ptr(pay["k_scale"]),
         _ptr(pay["qk_corr"]), _ptr(v_fp8_t), _ptr(v_scale), _ptr(v_mean), _ptr(out),
         _DT[out.dtype], B, H, N, d, int(bool(causal)), float(sm_scale),
-        _QKF[_qk_bits_of(pay["q_i4"])], _stream(out))
+        _format_of(pay), _stream(out))
     _check("sage2_attn_fwd_quantized_ex", st)
     return out
 
@@ -216,12 +244,11 @@ def sage2_attn_fwd_quantized(pay: dict, v_fp8_t: torch.Tensor, v_scale: torch.Te
 def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                    sm_scale: float | None = None, out_dtype=None,
                    out: torch.Tensor | None = None, qk_bits: int = 4,
-                   smooth_v: bool = False) -> torch.Tensor:
+                   smooth_v: bool = False, packed: bool = False) -> torch.Tensor:
     """Full forward pass (quantization + correction + attention) on q's stream.
     qk_bits 4 is the method (INT4 Q/K); 8 is the INT8 variant.  smooth_v turns
-    on V smoothing."""
-    if qk_bits not in _QKF:
-        raise ValueError("qk_bits must be 4 or 8")
+    on V smoothing; packed stores the INT4 payloads two per byte."""
+    fmt = _fmt(qk_bits, packed)
     B, H, N, d = _dims(q)
     for t in (k, v):
         if t.shape != q.shape or t.dtype != q.dtype:
@@ -233,7 +260,7 @@ def sage2_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bo
         out = torch.empty(B, H, N, d, dtype=out_dtype or q.dtype, device=q.device)
     st = lib().sage2_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, _DT[q.dtype],
                                  _DT[out.dtype], int(bool(causal)), float(sm_scale),
-                                 _QKF[qk_bits], int(bool(smooth_v)), _stream(q))
+                                 fmt, int(bool(smooth_v)), _stream(q))
     _check("sage2_attn_fwd_ex", st)
     return out
 

@@ -107,8 +107,11 @@ static sage2_status check_ptrs(P... ps) {
   return SAGE2_OK;
 }
 
-static bool valid_qk_format(int f) { return f == SAGE2_QK_INT4 || f == SAGE2_QK_INT8; }
+static bool valid_qk_format(int f) {
+  return f == SAGE2_QK_INT4 || f == SAGE2_QK_INT8 || f == SAGE2_QK_INT4_PACKED;
+}
 static int qk_bits_of(int f) { return f == SAGE2_QK_INT8 ? 8 : 4; }
+static bool packed_of(int f) { return f == SAGE2_QK_INT4_PACKED; }
 
 static sage2_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return SAGE2_OK;
@@ -119,12 +122,14 @@ static sage2_status from_cuda(cudaError_t e) {
 // ------------------------------------------------------------ workspace
 struct Workspace {
   size_t off_q_i4, off_k_i4, off_vt, off_qs, off_ks, off_qm, off_km, off_corr, off_vs, off_part,
-      off_amax, off_qsplit, off_vmean, total;
+      off_amax, off_qsplit, off_vmean, off_qpk, off_kpk, total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-static Workspace layout(const Dims& g) {
+// packed: room for the packed INT4 payloads as well (SAGE2_QK_INT4_PACKED),
+// which the quantizer writes and an unpack pass expands into q_i4 / k_i4.
+static Workspace layout(const Dims& g, bool packed = false) {
   Workspace w{};
   const size_t BH = static_cast<size_t>(g.BH), Np = g.Np, NB = g.NB, d = g.d;
   size_t o = 0;
@@ -146,6 +151,8 @@ static Workspace layout(const Dims& g) {
   w.off_amax = take(BH * d * 4);
   w.off_qsplit = take(3 * BH * ((NB + 127) / 128) * 128 * d * 2);
   w.off_vmean = take(BH * d * 4);
+  w.off_qpk = packed ? take(BH * Np * d / 2) : 0;
+  w.off_kpk = packed ? take(BH * Np * d / 2) : 0;
   w.total = o;
   return w;
 }
@@ -173,10 +180,12 @@ static cudaMemPool_t device_pool(int dev) {
 // One forward pass over B*H heads of N tokens: q/k/v heads ldh tokens apart,
 // o heads ldo tokens apart, payloads in the workspace ws (layout(g)), all on st.
 static cudaError_t forward(const void* q, const void* k, const void* v, void* o, const Dims& g,
-                           int dtype, int o_dtype, int causal, float sm_scale, int qk_bits,
+                           int dtype, int o_dtype, int causal, float sm_scale, int qk_format,
                            int smooth_v, int64_t ldh, int64_t ldo, uint8_t* ws, cudaStream_t st) {
   const int B = g.B, H = g.H, N = g.N, d = g.d;
-  const Workspace w = layout(g);
+  const int qk_bits = qk_bits_of(qk_format);
+  const bool packed = packed_of(qk_format);
+  const Workspace w = layout(g, packed);
   cudaError_t e;
   uint8_t* q_i4 = reinterpret_cast<uint8_t*>(ws + w.off_q_i4);
   uint8_t* k_i4 = reinterpret_cast<uint8_t*>(ws + w.off_k_i4);
@@ -191,13 +200,19 @@ static cudaError_t forward(const void* q, const void* k, const void* v, void* o,
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
   float* vmean = smooth_v ? reinterpret_cast<float*>(ws + w.off_vmean) : nullptr;
 
-  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, qs, qm, k_i4, ks, km, corr, part,
-            ws + w.off_qsplit, causal, qk_bits, ldh};
+  QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, packed ? ws + w.off_qpk : q_i4, qs, qm,
+            packed ? ws + w.off_kpk : k_i4, ks, km, corr, part, ws + w.off_qsplit, causal, qk_bits,
+            ldh, packed ? 1 : 0};
   // the V mean reuses the K-mean scratch: stream order puts it after the K mean
   VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, vmean, part, ldh};
   AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
               sm_scale, qk_bits, vmean, ldo};
   e = launch_smooth_quant_qk(qa, st);
+  if (e == cudaSuccess && packed) {
+    const size_t pk_bytes = static_cast<size_t>(g.BH) * g.Np * d / 2;
+    e = launch_unpack_int4(ws + w.off_qpk, q_i4, pk_bytes, st);
+    if (e == cudaSuccess) e = launch_unpack_int4(ws + w.off_kpk, k_i4, pk_bytes, st);
+  }
   if (e == cudaSuccess) e = launch_quant_v(va, st);
   if (e == cudaSuccess) e = launch_attn(aa, st);
   return e;
@@ -217,6 +232,8 @@ sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, i
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;
   if (dtype != SAGE2_F16 && dtype != SAGE2_BF16) return SAGE2_ERR_INVALID_ARG;
+  const int causal_corr = (qk_format & SAGE2_QK_CAUSAL_CORR) ? 1 : 0;
+  qk_format &= ~SAGE2_QK_CAUSAL_CORR;
   if (!valid_qk_format(qk_format)) return SAGE2_ERR_INVALID_ARG;
   s = check_ptrs(q, k, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
   if (s != SAGE2_OK) return s;
@@ -234,8 +251,8 @@ sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, i
                                           part_bytes + split_bytes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
   QKArgs a{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean,
-           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, 0,
-           qk_bits_of(qk_format), static_cast<int64_t>(N)};
+           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, causal_corr,
+           qk_bits_of(qk_format), static_cast<int64_t>(N), packed_of(qk_format) ? 1 : 0};
   e = launch_smooth_quant_qk(a, st);
   const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
@@ -304,7 +321,25 @@ sage2_status sage2_attn_fwd_quantized_ex(const uint8_t* q_i4, const float* q_sca
   AttnArgs a{q_i4, q_scale, k_i4, k_scale, qk_corr, v_fp8_t, v_scale, o, o_dtype,
              B,    H,       N,    d,       g.Np,    g.NB,    causal,  sm_scale,
              qk_bits_of(qk_format), v_mean, static_cast<int64_t>(N)};
-  return from_cuda(launch_attn(a, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!packed_of(qk_format)) return from_cuda(launch_attn(a, st));
+  // packed INT4: expand both payloads to e4m3 codes in pool scratch first
+  const size_t codes = up256(static_cast<size_t>(g.BH) * g.Np * d);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE2_ERR_CUDA;
+  cudaMemPool_t pool = device_pool(dev);
+  if (!pool) return SAGE2_ERR_CUDA;
+  uint8_t* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch), 2 * codes, pool, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  e = launch_unpack_int4(q_i4, scratch, static_cast<size_t>(g.BH) * g.Np * d / 2, st);
+  if (e == cudaSuccess)
+    e = launch_unpack_int4(k_i4, scratch + codes, static_cast<size_t>(g.BH) * g.Np * d / 2, st);
+  a.q_i4 = scratch;
+  a.k_i4 = scratch + codes;
+  if (e == cudaSuccess) e = launch_attn(a, st);
+  const cudaError_t e2 = cudaFreeAsync(scratch, st);
+  return from_cuda(e != cudaSuccess ? e : e2);
 }
 
 sage2_status sage2_attn_fwd_quantized(const uint8_t* q_i4, const float* q_scale,
@@ -345,12 +380,12 @@ sage2_status sage2_attn_fwd_ex(const void* q, const void* k, const void* v, void
   if (e != cudaSuccess) return SAGE2_ERR_CUDA;
   cudaMemPool_t pool = device_pool(dev);
   if (!pool) return SAGE2_ERR_CUDA;
-  const Workspace w = layout(g);
+  const Workspace w = layout(g, packed_of(qk_format));
   uint8_t* ws = nullptr;
   e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), w.total, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
 
-  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, qk_bits_of(qk_format), smooth_v,
+  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, qk_format, smooth_v,
               static_cast<int64_t>(N), static_cast<int64_t>(N), ws, st);
   const cudaError_t e2 = cudaFreeAsync(ws, st);
   return from_cuda(e != cudaSuccess ? e : e2);
@@ -365,7 +400,7 @@ sage2_status sage2_attn_fwd(const void* q, const void* k, const void* v, void* o
 
 sage2_status sage2_debug_qk_s32_ex(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int N,
                                    int d, int qk_format, int32_t* s_out, sage2_stream_t stream) {
-  if (!valid_qk_format(qk_format)) return SAGE2_ERR_INVALID_ARG;
+  if (!valid_qk_format(qk_format) || packed_of(qk_format)) return SAGE2_ERR_INVALID_ARG;
   Dims g;
   sage2_status s = check_dims(B, H, N, d, &g);
   if (s != SAGE2_OK) return s;

@@ -195,6 +195,14 @@ __global__ void __launch_bounds__(256, 1)
     for (int i = 0; i < ntiles; ++i) {
       const int s = i & 1;
       if (!mbar_wait_warp(&sm.d_full[s], (i >> 1) & 1, abort_flag)) break;
+      // causal: block rows before the key tile never read it; this warp's 32
+      // rows are all before it when its last row is
+      if (skip_masked && kt0 + i > row0 + 31) {
+        tc_fence_before();
+        __syncwarp();
+        mbar_arrive_lane0(&sm.d_empty[s], lane);
+        continue;
+      }
       tc_fence_after();
       uint32_t v[4][32];
       tmem_ld32(tmem + s * 128 + lane_off + 0, v[0]);

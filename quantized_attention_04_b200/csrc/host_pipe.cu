@@ -74,7 +74,7 @@ extern "C" sage2_status sage2_attn_fwd_host(const void* q, const void* k, const 
   if (s != SAGE2_OK) return s;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t in_bytes = up(per_chunk * head_in), out_bytes = up(per_chunk * head_out);
-  const size_t lane_bytes = 3 * in_bytes + out_bytes + up(layout(gc).total);
+  const size_t lane_bytes = 3 * in_bytes + out_bytes + up(layout(gc, packed_of(qk_format)).total);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int dev = 0;
@@ -90,7 +90,6 @@ extern "C" sage2_status sage2_attn_fwd_host(const void* q, const void* k, const 
   e = cudaEventRecord(lanes->fork, st);
   for (int i = 0; e == cudaSuccess && i < nlanes; ++i) e = cudaStreamWaitEvent(lanes->s[i], lanes->fork, 0);
 
-  const int qk_bits = qk_bits_of(qk_format);
   for (int64_t c = 0; e == cudaSuccess && c < nchunks; ++c) {
     const int lane = static_cast<int>(c % nlanes);
     cudaStream_t ls = lanes->s[lane];
@@ -108,7 +107,7 @@ extern "C" sage2_status sage2_attn_fwd_host(const void* q, const void* k, const 
     if (e != cudaSuccess) break;
     Dims gh;
     check_dims(1, nh, N, d, &gh);                                          // nh <= per_chunk: valid
-    e = forward(dq, dk, dv, dout, gh, dtype, o_dtype, causal, sm_scale, qk_bits, smooth_v,
+    e = forward(dq, dk, dv, dout, gh, dtype, o_dtype, causal, sm_scale, qk_format, smooth_v,
                 static_cast<int64_t>(N), static_cast<int64_t>(N), ws, ls);
     if (e == cudaSuccess)
       e = cudaMemcpyAsync(static_cast<uint8_t*>(o) + h0 * head_out, dout, ob, cudaMemcpyDeviceToHost, ls);

@@ -88,7 +88,7 @@ extern "C" sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, con
   if (ws == nullptr) return SAGE2_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, 4, 0, static_cast<int64_t>(N),
+  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, SAGE2_QK_INT4, 0, static_cast<int64_t>(N),
               static_cast<int64_t>(N), ws, st);
   return from_cuda(e);
 }

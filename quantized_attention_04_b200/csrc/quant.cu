@@ -108,12 +108,14 @@ __global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int
 // ---------------------------------------------------------------------------
 // Smoothing + INT4.  grid (NB, B*H, 2): z = 0 quantizes the Q block (after
 // computing its mean), z = 1 the K block (after subtracting kbar).  256 threads.
+// FMT: 0 INT4 values as e4m3 codes, 1 INT8 values (the variant), 2 INT4 values
+// packed two per byte (two's-complement nibbles, channel 2c in bits 3:0).
 // Two lanes own one row (16 rows per warp), each half of its channels, so a
 // row's amax needs one shuffle and its scale none.  In shared memory row r
 // starts at byte RS*r and its second half at +HO (RS = 2D+32, HO = D+16): the
 // 16-byte chunks that the eight lanes of one access phase read then fall in
 // eight different bank groups.
-template <typename T, int D, bool Q8>
+template <typename T, int D, int FMT>
 __global__ void __launch_bounds__(256) k_smooth_quant(
     const T* __restrict__ q, const T* __restrict__ k, int N, long long ldh, int Np, int NB,
     const float* __restrict__ kmean, uint8_t* __restrict__ q_i4, float* __restrict__ q_scale,
@@ -129,15 +131,19 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   const int r0 = blk * 128;
   const int nvalid = min(128, N - r0);
 
-  // coalesced 16-byte loads of the valid rows
+  // coalesced 16-byte asynchronous copies of the valid rows, all in flight at once
   const uint4* g = reinterpret_cast<const uint4*>(src + ((size_t)bh * ldh + r0) * D);
-  for (int i = threadIdx.x; i < nvalid * CPR; i += 256) {
+  constexpr int kPer = 128 * CPR / 256;            // copies per thread for a full block
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + 256 * u;
     const int r = i / CPR, j = i % CPR;
-    *reinterpret_cast<uint4*>(tile + RS * r + (j < CPH ? 16 * j : HO + 16 * (j - CPH))) = __ldg(g + i);
+    if (r < nvalid) cp_async16(tile + RS * r + (j < CPH ? 16 * j : HO + 16 * (j - CPH)), g + i);
   }
+  cp_async_wait_all();
 
+  __syncthreads();
   if (is_q) {
-    __syncthreads();
     if (threadIdx.x < D) {
       const int c = threadIdx.x;
       const int off = c < D / 2 ? 2 * c : HO + 2 * (c - D / 2);
@@ -156,7 +162,9 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   }
   __syncthreads();
 
-  uint8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * D;
+  constexpr bool Q8 = FMT == 1;
+  constexpr int RB = FMT == 2 ? D / 2 : D;        // payload bytes per row
+  uint8_t* out = (is_q ? q_i4 : k_i4) + ((size_t)bh * Np + r0) * RB;
   float* scale = (is_q ? q_scale : k_scale) + (size_t)bh * Np + r0;
   constexpr float kQmax = Q8 ? 127.f : 7.f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   // .16x256b TMEM loads then give each thread 32 consecutive keys).  Q^ rows
   // keep their natural order.
   const int srow = is_q ? r : 8 * ((r >> 1) & 15) + 2 * (r >> 5) + (r & 1);
-  uint8_t* orow = out + (size_t)srow * D + (D / 2) * hh;
+  uint8_t* orow = out + (size_t)srow * RB + (RB / 2) * hh;
   // Pass 2: quantize.  |x| <= amax and inv = RN(qmax/amax), so |x*inv| <=
   // qmax*(1+2^-24)^2 < qmax + 1/2: the rounded value never leaves [-qmax,
   // qmax] and needs no clamp.  Adding +0 turns a rounded -0 into +0 (the
@@ -208,6 +216,30 @@ __global__ void __launch_bounds__(256) k_smooth_quant(
   // the INT4 values exactly (at the same rate as the 8-bit integer path) and
   // yields S as an fp32 integer.  Zero is stored as +0 (code 0x00).
   // INT8 (the variant): values in [-127, 127] as two's-complement bytes.
+  if (FMT == 2) {
+    // two values per byte: 16 channels of this lane's half -> 8 bytes
+#pragma unroll
+    for (int i = 0; i < CPH; i += 2) {
+      uint32_t w[2] = {0u, 0u};
+      if (nz) {
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          float x[8];
+          load8(i + c2, x);
+#pragma unroll
+          for (int u = 0; u < 8; u += 2) {
+            const float2 p = __fmul2_rn(make_float2(x[u], x[u + 1]), inv2);
+            const uint32_t n0 = static_cast<uint32_t>(static_cast<int>(rintf(p.x))) & 0xFu;
+            const uint32_t n1 = static_cast<uint32_t>(static_cast<int>(rintf(p.y))) & 0xFu;
+            w[c2] |= (n0 | (n1 << 4)) << (4 * u);
+          }
+        }
+      }
+      *reinterpret_cast<uint2*>(orow + 4 * i) = make_uint2(w[0], w[1]);
+    }
+    if (hh == 0) scale[r] = sc;
+    return;
+  }
 #pragma unroll
   for (int i = 0; i < CPH; i += 2) {
     uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -305,7 +337,13 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
   constexpr int VPR = D / 8;
   const uint4* g = reinterpret_cast<const uint4*>(v + ((size_t)bh * ldh + t0) * D);
   uint4* s = reinterpret_cast<uint4*>(&tile[0][0]);
-  for (int i = threadIdx.x; i < nvalid * VPR; i += 256) s[i] = __ldg(g + i);
+  // asynchronous 16-byte copies, all of a thread's in flight at once
+#pragma unroll
+  for (int u = 0; u < 128 * VPR / 256; ++u) {
+    const int i = threadIdx.x + 256 * u;
+    if (i < nvalid * VPR) cp_async16(s + i, g + i);
+  }
+  cp_async_wait_all();
   if (threadIdx.x < D) {
     const float a = __uint_as_float(amax_bits[(size_t)bh * D + threadIdx.x]);
     inv[threadIdx.x] = a > 0.f ? __fdiv_rn(448.f, a) : 0.f;
@@ -342,6 +380,47 @@ __global__ void __launch_bounds__(256) k_v_quant(const T* __restrict__ v, int N,
 }
 
 // ---------------------------------------------------------------------------
+// Packed INT4 -> e4m3 codes, for the tensor path (B200 multiplies no INT4
+// operands; the INT4 values travel as e4m3 codes, exact for [-7, 7]).  A
+// 256-entry table maps a packed byte to its two codes, built from the same
+// conversion the quantizer uses.  Each thread expands 8 bytes into 16 codes.
+__global__ void __launch_bounds__(256) k_unpack_int4(const uint2* __restrict__ pk,
+                                                     uint4* __restrict__ codes, size_t n8) {
+  __shared__ uint32_t lut[256];
+  {
+    const int b = threadIdx.x;
+    const int lo = (b & 0xF) - ((b & 0x8) << 1);
+    const int hi = ((b >> 4) & 0xF) - ((b & 0x80) >> 3);
+    const uint32_t clo = __nv_cvt_float_to_fp8(static_cast<float>(lo), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t chi = __nv_cvt_float_to_fp8(static_cast<float>(hi), __NV_SATFINITE, __NV_E4M3);
+    lut[b] = clo | (chi << 8);
+  }
+  __syncthreads();
+  for (size_t i = static_cast<size_t>(blockIdx.x) * 256 + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * 256) {
+    const uint2 w = __ldg(pk + i);
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t src = j < 2 ? w.x : w.y;
+      const int sh = (j & 1) * 16;
+      o[j] = lut[(src >> sh) & 0xFFu] | (lut[(src >> (sh + 8)) & 0xFFu] << 16);
+    }
+    codes[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+cudaError_t launch_unpack_int4(const uint8_t* packed, uint8_t* codes, size_t bytes, cudaStream_t st) {
+  const size_t n8 = bytes / 8;
+  if (n8 == 0) return cudaSuccess;
+  const size_t want = (n8 + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
+  k_unpack_int4<<<grid, 256, 0, st>>>(reinterpret_cast<const uint2*>(packed),
+                                      reinterpret_cast<uint4*>(codes), n8);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Host-side launchers (called by the C ABI after validation).
 template <typename T, int D>
 cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st);  // corr.cu
@@ -355,11 +434,15 @@ static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
       static_cast<const T*>(a.k), a.N, a.ldh, nchunks, a.mean_part);
   k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, nchunks, a.N, D, a.k_mean);
   if (a.qk_bits == 8)
-    k_smooth_quant<T, D, true><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
+    k_smooth_quant<T, D, 1><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
+        a.q_scale, a.q_mean, a.k_i4, a.k_scale);
+  else if (a.packed)
+    k_smooth_quant<T, D, 2><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
         a.q_scale, a.q_mean, a.k_i4, a.k_scale);
   else
-    k_smooth_quant<T, D, false><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
+    k_smooth_quant<T, D, 0><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
         a.q_scale, a.q_mean, a.k_i4, a.k_scale);
   cudaError_t e = cudaGetLastError();

@@ -25,6 +25,7 @@ struct QKArgs {
   int skip_masked_corr;    // 1: skip correction blocks a causal mask hides
   int qk_bits;             // 4: INT4 values as e4m3 codes; 8: INT8 values (two's complement)
   int64_t ldh;             // tokens between consecutive heads of q and k (N when contiguous)
+  int packed;              // 1 (with qk_bits 4): q_i4/k_i4 hold two INT4 nibbles per byte
 };
 
 struct VArgs {
@@ -61,6 +62,9 @@ cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const VArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_debug_wait_timeout(cudaStream_t st);
+// Packed INT4 (two two's-complement nibbles per byte, channel 2c in bits 3:0)
+// -> one e4m3 code per value; `bytes` packed bytes, a multiple of 8.
+cudaError_t launch_unpack_int4(const uint8_t* packed, uint8_t* codes, size_t bytes, cudaStream_t st);
 cudaError_t launch_debug_qk(const uint8_t* q_i4, const uint8_t* k_i4, int B, int H, int Np, int d,
                             int qk_bits, int32_t* s_out, cudaStream_t st);
 

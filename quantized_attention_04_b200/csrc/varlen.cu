@@ -104,7 +104,7 @@ extern "C" sage2_status sage2_attn_fwd_varlen(const void* q, const void* k, cons
   nlanes = std::min(nlanes, kVarlenStreams);
   if (nlanes == 0) return SAGE2_OK;
 
-  const size_t ws_bytes = (layout(gmax).total + 255) & ~static_cast<size_t>(255);
+  const size_t ws_bytes = (layout(gmax, packed_of(qk_format)).total + 255) & ~static_cast<size_t>(255);
   uint8_t* ws = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), ws_bytes * nlanes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
@@ -128,7 +128,7 @@ extern "C" sage2_status sage2_attn_fwd_varlen(const void* q, const void* k, cons
     e = forward(static_cast<const uint8_t*>(q) + t0 * in_row,
                 static_cast<const uint8_t*>(k) + t0 * in_row,
                 static_cast<const uint8_t*>(v) + t0 * in_row, static_cast<uint8_t*>(o) + t0 * out_row,
-                g, dtype, o_dtype, causal, sm_scale, qk_bits_of(qk_format), smooth_v,
+                g, dtype, o_dtype, causal, sm_scale, qk_format, smooth_v,
                 static_cast<int64_t>(T), static_cast<int64_t>(T), ws + lane * ws_bytes,
                 lanes->s[lane]);
   }

@@ -154,6 +154,14 @@ def int4_codes(i) -> np.ndarray:
     return orc.e4m3_encode(np.asarray(i, np.float64))
 
 
+def pack_int4(values) -> np.ndarray:
+    """The library's packed INT4 layout (SAGE2_QK_INT4_PACKED): [..., d] INT4
+    values -> [..., d/2] bytes, channel 2c in bits 3:0 and 2c+1 in bits 7:4 of
+    byte c, each a two's-complement nibble."""
+    v = np.asarray(values, np.int64) & 0xF
+    return (v[..., 0::2] | (v[..., 1::2] << 4)).astype(np.uint8)
+
+
 def int4_values(codes) -> np.ndarray:
     """INT4 values back from the library's e4m3 codes (must be integers in [-7, 7])."""
     v = orc.e4m3_decode(np.asarray(codes, np.uint8))

@@ -95,13 +95,17 @@ def test_validation_variant_entries(L):
         a.update(kw)
         return L.sage2_attn_fwd_ex(a["q"], a["k"], a["v"], a["o"], a["B"], a["H"], a["N"], a["d"],
                                    a["dt"], a["odt"], a["causal"], a["sm"], fmt, smooth, None)
-    assert attn_ex(fmt=2) == 1
+    assert attn_ex(fmt=3) == 1
     assert attn_ex(fmt=-1) == 1
+    assert attn_ex(fmt=2, d=96) == 2               # packed INT4 is a valid format
+    assert attn_ex(fmt=2, q=P + 4) == 3
     assert attn_ex(smooth=2) == 1
     assert attn_ex(fmt=1, d=96) == 2
     assert attn_ex(fmt=1, q=P + 4) == 3
     z = [P] * 7
     assert L.sage2_smooth_quant_qk_ex(P, P, 0, 1, 1, 10, 64, *z, 3, None) == 1
+    assert L.sage2_smooth_quant_qk_ex(P, P, 0, 1, 1, 10, 64, *z, 0x100 | 3, None) == 1
+    assert L.sage2_smooth_quant_qk_ex(P, P, 0, 1, 1, 10, 96, *z, 0x100 | 2, None) == 2
     assert L.sage2_smooth_quant_qk_ex(P, P, 0, 1, 1, 0, 64, *z, 1, None) == 1
     assert L.sage2_quant_v_ex(P, 0, 1, 1, 10, 64, P, P, P + 8, None) == 3     # misaligned v_mean
     assert L.sage2_quant_v_ex(P, 0, 1, 1, 10, 64, P, 0, P, None) == 1
@@ -110,6 +114,7 @@ def test_validation_variant_entries(L):
     assert L.sage2_attn_fwd_quantized_ex(P, P, P, P, P, P, P, P + 4, P, 2, 1, 1, 10, 64, 0, 0.1, 1,
                                          None) == 3
     assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 7, P, None) == 1
+    assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 2, P, None) == 1   # packed: not here
     assert L.sage2_debug_qk_s32_ex(P, P, 1, 1, 10, 64, 1, 0, None) == 1
 
 

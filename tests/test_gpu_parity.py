@@ -136,6 +136,28 @@ def test_attention_quantized_entry_matches_full(qa):
     assert torch.equal(o1, o2)
 
 
+def test_causal_correction_flag(qa):
+    """With SAGE2_QK_CAUSAL_CORR the correction entries a causal attention reads
+    (key tile <= query block) are those of the full write, bit for bit, and the
+    causal attention over them gives the same output."""
+    cfg = small_cfg(1000, 128, "bf16", True)
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    sm = P.default_scale(cfg.d)
+    full = qa.sage2_smooth_quant_qk(qd, kd)
+    part = qa.sage2_smooth_quant_qk(qd, kd, causal_corr=True)
+    vt, vs = qa.sage2_quant_v(vd)
+    o1 = qa.sage2_attn_fwd_quantized(full, vt, vs, cfg.N, True, sm, torch.float32)
+    o2 = qa.sage2_attn_fwd_quantized(part, vt, vs, cfg.N, True, sm, torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    nb = orc.n_pad(cfg.N) // 128
+    cf, cp = full["qk_corr"].cpu().numpy(), part["qk_corr"].cpu().numpy()
+    for blk in range(nb):
+        assert P.bits_equal(cp[:, :, blk, :(blk + 1) * 128], cf[:, :, blk, :(blk + 1) * 128]), blk
+    for n in ("q_i4", "q_scale", "q_mean", "k_i4", "k_scale", "k_mean"):
+        assert torch.equal(full[n], part[n]), n
+
+
 @pytest.mark.parametrize("name", ["C2"])
 def test_attention_config_full(qa, name):
     cfg = CONFIGS[name]

@@ -1,6 +1,7 @@
-"""GPU parity of the two variants (NEXT rows of the scope table) against the
+"""GPU parity of the variants (NEXT rows of the scope table) against the
 CPU oracle, through the C ABI: INT8 Q/K (payload format SAGE2_QK_INT8, the
-8-bit integer tensor path) and V smoothing.  Same tolerances as the method's
+8-bit integer tensor path), V smoothing, and INT4 stored two per byte
+(SAGE2_QK_INT4_PACKED).  Same tolerances as the method's
 own parity tests (tests/parity.py): payloads bit-exact, O within 2e-3 /
 rel-L1 1e-3 after the oracle's ambiguity bound."""
 import numpy as np
@@ -152,3 +153,54 @@ def test_variants_config_sampled(qa, name):
         P.assert_o_close(P.np32(o[b, h])[rows], O, amb, cfg.torch_dtype,
                          flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows, what=
                          (name, qk_bits, smooth_v))
+
+
+# ------------------------------------------------------- packed INT4 (2 per byte)
+@pytest.mark.parametrize("cfg", SMALL + [CONFIGS["C1"]], ids=lambda c: c.name)
+def test_packed_int4_payloads_bit_exact(qa, cfg):
+    """The oracle's INT4 values, packed by the test helper, against the
+    library's packed payloads (k rows in the library's permuted order)."""
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    pay = qa.sage2_smooth_quant_qk(qd, kd, packed=True)
+    torch.cuda.synchronize()
+    assert pay["q_i4"].shape[-1] * 2 == cfg.d
+    g = {n: t.cpu().numpy() for n, t in pay.items()}
+    Np = orc.n_pad(cfg.N)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            o = orc.smooth_quant_qk(P.np32(q[b, h]), P.np32(k[b, h]))
+            o["k_i4"] = o["k_i4"][P.key_interleave(Np)]
+            assert np.array_equal(g["q_i4"][b, h], P.pack_int4(o["q_i4"])), (b, h)
+            assert np.array_equal(g["k_i4"][b, h], P.pack_int4(o["k_i4"])), (b, h)
+            for name in ("q_scale", "q_mean", "k_scale", "k_mean"):
+                assert P.bits_equal(g[name][b, h], o[name]), (name, b, h)
+
+
+@pytest.mark.parametrize("cfg", SMALL + [CONFIGS["C1"]], ids=lambda c: c.name)
+def test_packed_int4_output_equals_int4(qa, cfg):
+    """The same INT4 values, stored packed, give the INT4 path's output bit for
+    bit: through the full call and through the stage calls."""
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    sm = P.default_scale(cfg.d)
+    o4 = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out_dtype=torch.float32)
+    op = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, out_dtype=torch.float32,
+                           packed=True)
+    pay = qa.sage2_smooth_quant_qk(qd, kd, packed=True)
+    vt, vs = qa.sage2_quant_v(vd)
+    os_ = qa.sage2_attn_fwd_quantized(pay, vt, vs, cfg.N, cfg.causal, sm, torch.float32)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    assert torch.equal(o4, op)
+    assert torch.equal(o4, os_)
+
+
+def test_packed_int4_config_sampled(qa):
+    """C3 at full size with packed payloads: the INT4 output, bit for bit."""
+    cfg = CONFIGS["C3"]
+    q, k, v, qd, kd, vd = _cuda(cfg)
+    sm = P.default_scale(cfg.d)
+    o4 = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm)
+    op = qa.sage2_attn_fwd(qd, kd, vd, causal=cfg.causal, sm_scale=sm, packed=True)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    assert torch.equal(o4, op)

@@ -58,3 +58,10 @@ def test_p_store_and_pv_k_order_match_the_value_map():
     assert sorted(k_index_token.tolist()) == list(range(128))
     # V^T byte p of a block must hold the token that K index p multiplies
     assert (k_index_token == P.value_interleave(128)).all()
+
+
+def test_packed_int4_layout_golden():
+    """Two INT4 values per byte, low nibble first, two's complement: hand-worked
+    bytes (1 | -1 << 4 = 0xF1, 7 | -7 << 4 = 0x97, -8 | 0 = 0x08, 0 | 3 = 0x30)."""
+    got = P.pack_int4(np.array([[1, -1, 7, -7, -8, 0, 0, 3]]))
+    assert got.tolist() == [[0xF1, 0x97, 0x08, 0x30]]
