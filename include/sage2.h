@@ -292,6 +292,12 @@ sage2_status sage2_debug_wait_timeout(sage2_stream_t stream);
  * Synchronizes `stream`, then reads and clears the device error word that
  * kernels set instead of trapping.  SAGE2_ERR_TIMEOUT if a bounded wait ran
  * out, SAGE2_ERR_CUDA on a sticky CUDA error, else SAGE2_OK.
+ * After SAGE2_ERR_TIMEOUT the outputs of the work enqueued since the last
+ * check are invalid (a block that gave up left its rows unwritten); the
+ * context stays usable and the call may simply be repeated.  A wait gives up
+ * after about one second of wall time, which a healthy launch can exceed only
+ * if the GPU stops running it for that long (for example a long preemption by
+ * another context on a shared GPU).
  */
 sage2_status sage2_check_device_error(sage2_stream_t stream);
 

@@ -14,8 +14,10 @@
 // with blocks on the M side (128 per chunk) and 128 keys on the N side.
 //
 // k_qbar_split : qbar -> three 16-bit terms, [3][B*H][NBc*128][d] (pad rows 0).
-// k_qk_corr_tc : one CTA = one head, one 128-block chunk, a run of key tiles.
-//   warp 0 TMA (the chunk's three term tiles once, then K tiles, 2 stages),
+// k_qk_corr_tc : persistent, one CTA per SM over a contiguous run of work items
+//   (head, 128-block chunk, key tile), in that order.
+//   warp 0 TMA (a chunk's three term tiles once per run of its items, then
+//   K tiles, 2 stages),
 //   warp 1 MMA issuer, warp 2 TMEM allocator, warps 4-7 epilogue: a warp owns
 //   32 block rows; per tile it stages four 32 x 32 fp32 boxes in shared memory
 //   (128-byte swizzle, conflict-free) and writes each with a TMA tensor store,
@@ -24,6 +26,7 @@
 //   load side, so their C is 0; the store clips block rows >= NB.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -32,8 +35,6 @@
 #include "sm100_ptx.cuh"
 
 namespace sage2 {
-
-constexpr int kCorrTilesPerCta = 8;
 
 template <typename T>
 struct IsBf16 {
@@ -79,7 +80,7 @@ struct __align__(1024) CorrSmem {
   uint8_t a[3][D / 64][128 * 128];   // term x 128-byte atom x (128 rows x 128 B)
   uint8_t b[2][D / 64][128 * 128];   // stage x atom: 128 keys x 64 channels
   uint8_t out[4][2][32 * 128];       // epilogue warp x buffer: 32 rows x 32 fp32 (swizzled)
-  uint64_t a_full;
+  uint64_t a_full, a_empty;
   uint64_t b_full[2], b_empty[2];
   uint64_t d_full[2], d_empty[2];
   uint64_t drain;
@@ -87,28 +88,50 @@ struct __align__(1024) CorrSmem {
   int abort_flag;
 };
 
+// Work item i (0 <= i < total) of a grid-wide list ordered by head, then
+// 128-block chunk, then key tile: the chunk's key tiles are 0 .. kt_end-1,
+// kt_end = NB, or with the causal skip the tiles up to the chunk's last block.
+struct CorrItem {
+  int bh, chunk, kt;
+};
+__device__ __forceinline__ int corr_tiles_of_chunk(int chunk, int NB, int skip_masked) {
+  return skip_masked ? min(NB, (chunk + 1) * 128) : NB;
+}
+__device__ __forceinline__ CorrItem corr_item(int i, int NB, int NBc, int per_head, int skip_masked) {
+  CorrItem it;
+  it.bh = i / per_head;
+  int r = i - it.bh * per_head;
+  int c = 0;
+  while (c + 1 < NBc && r >= corr_tiles_of_chunk(c, NB, skip_masked)) {
+    r -= corr_tiles_of_chunk(c, NB, skip_masked);
+    ++c;
+  }
+  it.chunk = c;
+  it.kt = r;
+  return it;
+}
+
+// Persistent: CTA c takes items [c*total/G, (c+1)*total/G); the three term
+// tiles of a (head, chunk) are loaded once per run of its items.
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 1)
     k_qk_corr_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_c, int N, int Np, int NB, int NBc,
-                 int BH, int skip_masked) {
+                 int BH, int skip_masked, int per_head, long long total) {
   extern __shared__ uint8_t smem_raw[];
   CorrSmem<D>& sm = *reinterpret_cast<CorrSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int kAtoms = D / 64;
   constexpr uint32_t kAtomBytes = 128 * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.y, bh = blockIdx.z;
-  // key tiles of this CTA; a causal mask hides keys beyond the chunk's last block
-  const int kt_end_all = skip_masked ? min(NB, (chunk + 1) * 128) : NB;
-  const int kt0 = blockIdx.x * kCorrTilesPerCta;
-  const int kt1 = min(kt_end_all, kt0 + kCorrTilesPerCta);
-  const int ntiles = kt1 - kt0;
-  if (ntiles <= 0) return;   // uniform across the block: before any barrier or TMEM use
+  const int i0 = static_cast<int>(total * blockIdx.x / gridDim.x);
+  const int i1 = static_cast<int>(total * (blockIdx.x + 1) / gridDim.x);
+  if (i1 <= i0) return;   // uniform across the block: before any barrier or TMEM use
   volatile int* abort_flag = &sm.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.a_full, 1);
+    mbar_init(&sm.a_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.b_full[s], 1);
       mbar_init(&sm.b_empty[s], 1);
@@ -132,28 +155,41 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_a);
       prefetch_tmap(&tm_k);
-      mbar_expect_tx(&sm.a_full, 3 * kAtoms * kAtomBytes);
-      for (int term = 0; term < 3; ++term)
-        for (int at = 0; at < kAtoms; ++at)
-          tma_load_2d(sm.a[term][at], &tm_a, &sm.a_full, 64 * at,
-                      (term * BH + bh) * NBc * 128 + chunk * 128);
-      int i = 0;
-      for (; i < ntiles; ++i) {
-        const int s = i & 1;
-        if (i >= 2 && !mbar_wait(&sm.b_empty[s], ((i >> 1) - 1) & 1, abort_flag)) break;
+      int g = -1, cur_bh = -1, cur_chunk = -1;
+      int i = i0;
+      bool ok = true;
+      for (; ok && i < i1; ++i) {
+        const CorrItem it = corr_item(i, NB, NBc, per_head, skip_masked);
+        if (it.bh != cur_bh || it.chunk != cur_chunk) {
+          // a new (head, chunk): its term tiles replace the previous ones once
+          // every MMA that read those has completed
+          ++g;
+          if (g >= 1 && !mbar_wait(&sm.a_empty, (g - 1) & 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&sm.a_full, 3 * kAtoms * kAtomBytes);
+          for (int term = 0; term < 3; ++term)
+            for (int at = 0; at < kAtoms; ++at)
+              tma_load_2d(sm.a[term][at], &tm_a, &sm.a_full, 64 * at,
+                          (term * BH + it.bh) * NBc * 128 + it.chunk * 128);
+          cur_bh = it.bh;
+          cur_chunk = it.chunk;
+        }
+        const int j = i - i0, s = j & 1;
+        if (j >= 2 && !mbar_wait(&sm.b_empty[s], ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(&sm.b_full[s], kAtoms * kAtomBytes);
         for (int at = 0; at < kAtoms; ++at) {
           asm volatile(
               "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
               " [%0], [%1, {%3, %4, %5}], [%2];"
               ::"r"(smem_u32(sm.b[s][at])), "l"(reinterpret_cast<uint64_t>(&tm_k)),
-                "r"(smem_u32(&sm.b_full[s])), "r"(64 * at), "r"((kt0 + i) * 128), "r"(bh)
+                "r"(smem_u32(&sm.b_full[s])), "r"(64 * at), "r"(it.kt * 128), "r"(it.bh)
               : "memory");
         }
       }
-      if (*abort_flag) {
-        mbar_wait(&sm.a_full, 0, nullptr);
-        for (int u = (i > 2 ? i - 2 : 0); u < i; ++u) mbar_wait(&sm.b_full[u & 1], (u >> 1) & 1, nullptr);
+      if (!ok) {
+        // let the copies already issued land before the block exits
+        if (g >= 0) mbar_wait(&sm.a_full, g & 1, nullptr);
+        const int n = i - i0;
+        for (int u = (n > 2 ? n - 2 : 0); u < n; ++u) mbar_wait(&sm.b_full[u & 1], (u >> 1) & 1, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -161,11 +197,19 @@ __global__ void __launch_bounds__(256, 1)
       constexpr uint32_t idesc = idesc_f16_f32(128, 128, IsBf16<T>::value);
       const uint64_t da = smem_desc_kmajor(sm.a[0][0], 128);
       const uint64_t db = smem_desc_kmajor(sm.b[0][0], 128);
-      bool ok = mbar_wait(&sm.a_full, 0, abort_flag);
-      for (int i = 0; ok && i < ntiles; ++i) {
-        const int s = i & 1;
-        if (!mbar_wait(&sm.b_full[s], (i >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(&sm.d_empty[s], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+      int g = -1, cur_bh = -1, cur_chunk = -1;
+      bool ok = true;
+      for (int i = i0; ok && i < i1; ++i) {
+        const CorrItem it = corr_item(i, NB, NBc, per_head, skip_masked);
+        if (it.bh != cur_bh || it.chunk != cur_chunk) {
+          ++g;
+          if (!mbar_wait(&sm.a_full, g & 1, abort_flag)) { ok = false; break; }
+          cur_bh = it.bh;
+          cur_chunk = it.chunk;
+        }
+        const int j = i - i0, s = j & 1;
+        if (!mbar_wait(&sm.b_full[s], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(&sm.d_empty[s], ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         int n = 0;
 #pragma unroll
@@ -180,6 +224,12 @@ __global__ void __launch_bounds__(256, 1)
         }
         tc_commit(&sm.d_full[s]);
         tc_commit(&sm.b_empty[s]);
+        // the last item of this (head, chunk): its term tiles may be replaced
+        // once these MMAs complete
+        if (i + 1 < i1) {
+          const CorrItem nx = corr_item(i + 1, NB, NBc, per_head, skip_masked);
+          if (nx.bh != cur_bh || nx.chunk != cur_chunk) tc_commit(&sm.a_empty);
+        }
       }
       if (!ok) {
         tc_commit(&sm.drain);
@@ -187,17 +237,18 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp >= 4) {
-    // epilogue: warp q owns block rows 32q..32q+31 of the chunk (its TMEM lanes)
+    // epilogue: warp q owns block rows 32q..32q+31 of the item's chunk (its TMEM lanes)
     const int q = warp - 4;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int row0 = chunk * 128 + q * 32;
     int nb = 0;                                          // staging buffer to fill next
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i & 1;
-      if (!mbar_wait_warp(&sm.d_full[s], (i >> 1) & 1, abort_flag)) break;
+    for (int i = i0; i < i1; ++i) {
+      const CorrItem it = corr_item(i, NB, NBc, per_head, skip_masked);
+      const int j = i - i0, s = j & 1;
+      const int row0 = it.chunk * 128 + q * 32;
+      if (!mbar_wait_warp(&sm.d_full[s], (j >> 1) & 1, abort_flag)) break;
       // causal: block rows before the key tile never read it; this warp's 32
       // rows are all before it when its last row is
-      if (skip_masked && kt0 + i > row0 + 31) {
+      if (skip_masked && it.kt > row0 + 31) {
         tc_fence_before();
         __syncwarp();
         mbar_arrive_lane0(&sm.d_empty[s], lane);
@@ -226,7 +277,7 @@ __global__ void __launch_bounds__(256, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tm_c, st, (kt0 + i) * 128 + 32 * grp, row0, bh);
+          tma_store_3d(&tm_c, st, it.kt * 128 + 32 * grp, row0, it.bh);
           bulk_commit();
         }
         nb ^= 1;
@@ -286,9 +337,19 @@ cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int groups = (a.NB + kCorrTilesPerCta - 1) / kCorrTilesPerCta;
-  k_qk_corr_tc<T, D><<<dim3(groups, NBc, BH), 256, smem, st>>>(
-      tma, tmk, tmc, a.N, a.Np, a.NB, NBc, BH, a.skip_masked_corr);
+  // items per head: each chunk's key tiles (all of them, or with the causal
+  // skip those up to the chunk's last block)
+  int per_head = 0;
+  for (int c = 0; c < NBc; ++c)
+    per_head += a.skip_masked_corr ? std::min(a.NB, (c + 1) * 128) : a.NB;
+  const long long total = static_cast<long long>(per_head) * BH;
+  if (total > INT32_MAX) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = std::min<long long>(total, sms);
+  k_qk_corr_tc<T, D><<<static_cast<unsigned>(grid), 256, smem, st>>>(
+      tma, tmk, tmc, a.N, a.Np, a.NB, NBc, BH, a.skip_masked_corr, per_head, total);
   return cudaGetLastError();
 }
 
