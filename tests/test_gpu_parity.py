@@ -120,8 +120,9 @@ def test_attention_small_full(qa, cfg, out_dtype):
     for b in range(cfg.B):
         for h in range(cfg.H):
             pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
-            P.assert_o_close(o[b, h][rows], O, amb, od, (cfg.name, b, h),
-                             flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
+            stats = P.assert_o_close(o[b, h][rows], O, amb, od, (cfg.name, b, h),
+                                     flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
+            print(cfg.name, od, (b, h), stats)
 
 
 def test_attention_quantized_entry_matches_full(qa):
@@ -169,8 +170,9 @@ def test_attention_config_full(qa, name):
     for b in range(cfg.B):
         for h in range(cfg.H):
             pay, O, amb, rows = P.oracle_head(q, k, v, b, h, cfg.causal, sm)
-            P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (name, b, h),
-                             flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
+            stats = P.assert_o_close(o[b, h][rows], O, amb, torch.float32, (name, b, h),
+                                     flips=P.head_flips(pay, cfg.N, cfg.causal, sm), rows=rows)
+            print(name, torch.float32, (b, h), stats)
 
 
 @pytest.mark.parametrize("out_dtype", ["input", torch.float32])
