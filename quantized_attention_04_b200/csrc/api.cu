@@ -122,7 +122,7 @@ static sage2_status from_cuda(cudaError_t e) {
 // ------------------------------------------------------------ workspace
 struct Workspace {
   size_t off_q_i4, off_k_i4, off_vt, off_qs, off_ks, off_qm, off_km, off_corr, off_vs, off_part,
-      off_amax, off_qsplit, off_vmean, off_qpk, off_kpk, total;
+      off_amax, off_qsplit, off_vmean, off_done, off_qpk, off_kpk, total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -151,6 +151,7 @@ static Workspace layout(const Dims& g, bool packed = false) {
   w.off_amax = take(BH * d * 4);
   w.off_qsplit = take(3 * BH * ((NB + 127) / 128) * 128 * d * 2);
   w.off_vmean = take(BH * d * 4);
+  w.off_done = take(2 * BH * 4);               // K-mean and V-mean block counters
   w.off_qpk = packed ? take(BH * Np * d / 2) : 0;
   w.off_kpk = packed ? take(BH * Np * d / 2) : 0;
   w.total = o;
@@ -177,11 +178,40 @@ static cudaMemPool_t device_pool(int dev) {
   return pools[dev];
 }
 
+// A library stream per device for running independent chains of one call
+// concurrently, with its fork / join events.  The lock is held while a call
+// enqueues (its events are recorded and waited on in that window).
+struct SideLane {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ok = false;
+};
+
+static SideLane* side_lane(int dev, std::unique_lock<std::mutex>* lock) {
+  static std::mutex mu[64];
+  static SideLane lanes[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  *lock = std::unique_lock<std::mutex>(mu[dev]);
+  SideLane& L = lanes[dev];
+  if (!L.ok) {
+    const bool good = cudaStreamCreateWithFlags(&L.s, cudaStreamNonBlocking) == cudaSuccess &&
+                      cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming) == cudaSuccess &&
+                      cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) == cudaSuccess;
+    if (!good) return nullptr;
+    L.ok = true;
+  }
+  return &L;
+}
+
 // One forward pass over B*H heads of N tokens: q/k/v heads ldh tokens apart,
 // o heads ldo tokens apart, payloads in the workspace ws (layout(g)), all on st.
+// With `side` (a SideLane held by the caller), the Q chain (Q smoothing,
+// q-mean split, correction) runs on the side stream while the K chain and the
+// V chain run on st; they join before the attention kernel.
 static cudaError_t forward(const void* q, const void* k, const void* v, void* o, const Dims& g,
                            int dtype, int o_dtype, int causal, float sm_scale, int qk_format,
-                           int smooth_v, int64_t ldh, int64_t ldo, uint8_t* ws, cudaStream_t st) {
+                           int smooth_v, int64_t ldh, int64_t ldo, uint8_t* ws, cudaStream_t st,
+                           SideLane* side = nullptr) {
   const int B = g.B, H = g.H, N = g.N, d = g.d;
   const int qk_bits = qk_bits_of(qk_format);
   const bool packed = packed_of(qk_format);
@@ -200,20 +230,26 @@ static cudaError_t forward(const void* q, const void* k, const void* v, void* o,
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws + w.off_amax);
   float* vmean = smooth_v ? reinterpret_cast<float*>(ws + w.off_vmean) : nullptr;
 
+  unsigned* done = reinterpret_cast<unsigned*>(ws + w.off_done);
   QKArgs qa{q, k, dtype, B, H, N, d, g.Np, g.NB, packed ? ws + w.off_qpk : q_i4, qs, qm,
             packed ? ws + w.off_kpk : k_i4, ks, km, corr, part, ws + w.off_qsplit, causal, qk_bits,
-            ldh, packed ? 1 : 0};
+            ldh, packed ? 1 : 0, done, side ? side->s : nullptr, side ? side->fork : nullptr,
+            nullptr};
   // the V mean reuses the K-mean scratch: stream order puts it after the K mean
-  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, vmean, part, ldh};
+  VArgs va{v, dtype, B, H, N, d, g.Np, g.NB, vt, vs, amax, vmean, part, ldh, done + g.BH};
   AttnArgs aa{q_i4, qs, k_i4, ks, corr, vt, vs, o, o_dtype, B, H, N, d, g.Np, g.NB, causal,
               sm_scale, qk_bits, vmean, ldo};
   e = launch_smooth_quant_qk(qa, st);
+  if (e == cudaSuccess) e = launch_quant_v(va, st);
+  if (e == cudaSuccess && side) {
+    e = cudaEventRecord(side->join, side->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
+  }
   if (e == cudaSuccess && packed) {
     const size_t pk_bytes = static_cast<size_t>(g.BH) * g.Np * d / 2;
     e = launch_unpack_int4(ws + w.off_qpk, q_i4, pk_bytes, st);
     if (e == cudaSuccess) e = launch_unpack_int4(ws + w.off_kpk, k_i4, pk_bytes, st);
   }
-  if (e == cudaSuccess) e = launch_quant_v(va, st);
   if (e == cudaSuccess) e = launch_attn(aa, st);
   return e;
 }
@@ -238,8 +274,9 @@ sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, i
   s = check_ptrs(q, k, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean, qk_corr);
   if (s != SAGE2_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // scratch: the K-mean partial sums and the split q_mean terms
+  // scratch: the K-mean partial sums and block counters, the split q_mean terms
   const size_t part_bytes = up256(static_cast<size_t>(g.BH) * g.NB * d * 4);
+  const size_t done_bytes = up256(static_cast<size_t>(g.BH) * 4);
   const size_t split_bytes =
       up256(3 * static_cast<size_t>(g.BH) * ((g.NB + 127) / 128) * 128 * d * 2);
   int dev = 0;
@@ -248,11 +285,16 @@ sage2_status sage2_smooth_quant_qk_ex(const void* q, const void* k, int dtype, i
   if (!pool) return SAGE2_ERR_CUDA;
   uint8_t* scratch = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch),
-                                          part_bytes + split_bytes, pool, st);
+                                          part_bytes + done_bytes + split_bytes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
+  // the Q chain runs on the library's side stream, concurrently with the K chain
+  std::unique_lock<std::mutex> lock;
+  SideLane* side = side_lane(dev, &lock);
   QKArgs a{q, k, dtype, B, H, N, d, g.Np, g.NB, q_i4, q_scale, q_mean, k_i4, k_scale, k_mean,
-           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes, causal_corr,
-           qk_bits_of(qk_format), static_cast<int64_t>(N), packed_of(qk_format) ? 1 : 0};
+           qk_corr, reinterpret_cast<float*>(scratch), scratch + part_bytes + done_bytes,
+           causal_corr, qk_bits_of(qk_format), static_cast<int64_t>(N),
+           packed_of(qk_format) ? 1 : 0, reinterpret_cast<unsigned*>(scratch + part_bytes),
+           side ? side->s : nullptr, side ? side->fork : nullptr, side ? side->join : nullptr};
   e = launch_smooth_quant_qk(a, st);
   const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
@@ -279,7 +321,9 @@ sage2_status sage2_quant_v_ex(const void* v, int dtype, int B, int H, int N, int
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // scratch: the per-channel |V| maximum and, with smoothing, the mean partial sums
   const size_t amax_bytes = up256(static_cast<size_t>(g.BH) * d * 4);
-  const size_t part_bytes = v_mean ? up256(static_cast<size_t>(g.BH) * g.NB * d * 4) : 0;
+  const size_t part_bytes = v_mean ? up256(static_cast<size_t>(g.BH) * g.NB * d * 4) +
+                                         up256(static_cast<size_t>(g.BH) * 4)
+                                   : 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE2_ERR_CUDA;
   cudaMemPool_t pool = device_pool(dev);
@@ -291,7 +335,10 @@ sage2_status sage2_quant_v_ex(const void* v, int dtype, int B, int H, int N, int
   VArgs a{v, dtype, B, H, N, d, g.Np, g.NB, v_fp8_t, v_scale,
           reinterpret_cast<uint32_t*>(scratch), v_mean,
           v_mean ? reinterpret_cast<float*>(scratch + amax_bytes) : nullptr,
-          static_cast<int64_t>(N)};
+          static_cast<int64_t>(N),
+          v_mean ? reinterpret_cast<unsigned*>(scratch + amax_bytes +
+                                               up256(static_cast<size_t>(g.BH) * g.NB * d * 4))
+                 : nullptr};
   e = launch_quant_v(a, st);
   const cudaError_t e2 = cudaFreeAsync(scratch, st);
   return from_cuda(e != cudaSuccess ? e : e2);
@@ -385,8 +432,12 @@ sage2_status sage2_attn_fwd_ex(const void* q, const void* k, const void* v, void
   e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), w.total, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
 
-  e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, qk_format, smooth_v,
-              static_cast<int64_t>(N), static_cast<int64_t>(N), ws, st);
+  {
+    std::unique_lock<std::mutex> lock;
+    SideLane* side = side_lane(dev, &lock);
+    e = forward(q, k, v, o, g, dtype, o_dtype, causal, sm_scale, qk_format, smooth_v,
+                static_cast<int64_t>(N), static_cast<int64_t>(N), ws, st, side);
+  }
   const cudaError_t e2 = cudaFreeAsync(ws, st);
   return from_cuda(e != cudaSuccess ? e : e2);
 }

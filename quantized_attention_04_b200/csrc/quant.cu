@@ -1,6 +1,6 @@
 // Smoothing and quantization kernels (HBM-bound passes).
 //
-//  k_mean_partial / k_mean_finalize : K smoothing - token mean of K per channel.
+//  k_mean_partial                   : K smoothing - token mean of K per channel.
 //  k_smooth_quant                   : Q smoothing (mean of each 128-row block) and
 //                                     K smoothing applied, then INT4 per token.
 //  (the correction qbar_blk . K_j added back to the INT4 product is in corr.cu)
@@ -51,63 +51,72 @@ __device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // ---------------------------------------------------------------------------
-// K mean, pass 1: one worker (D/8 threads, 8 channels each) per 128-token
-// chunk sums its chunk token by token in ascending order (fp32).
-// grid (ceil(nchunks / workers_per_block), B*H), 256 threads.
+// K mean: one worker (D/8 threads, 8 channels each) per 128-token chunk sums
+// its chunk token by token in ascending order (fp32) into part[bh][chunk].
+// The last block of a head to finish (a per-head counter) then adds the chunk
+// sums in chunk order and divides once by N (fp32), and resets the counter.
+// grid (ceil(nchunks / workers_per_block), B*H), 256 threads; done[] starts at 0.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_mean_partial(const T* __restrict__ k, int N,
                                                       long long ldh, int nchunks,
-                                                      float* __restrict__ part) {
+                                                      float* __restrict__ part,
+                                                      unsigned* __restrict__ done,
+                                                      float* __restrict__ kmean) {
   constexpr int TPR = D / 8;
   constexpr int WPB = 256 / TPR;
   const int bh = blockIdx.y;
   const int worker = threadIdx.x / TPR, q8 = threadIdx.x % TPR;
   const int chunk = blockIdx.x * WPB + worker;
-  if (chunk >= nchunks) return;
-  const int t0 = chunk * 128;
-  const int nt = min(128, N - t0);
-  const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bh * ldh + t0) * D) + q8;
-  float acc[8];
+  if (chunk < nchunks) {
+    const int t0 = chunk * 128;
+    const int nt = min(128, N - t0);
+    const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bh * ldh + t0) * D) + q8;
+    float acc[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  int t = 0;
-  for (; t + 8 <= nt; t += 8) {
-    uint4 u[8];
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    int t = 0;
+    for (; t + 8 <= nt; t += 8) {
+      uint4 u[8];
 #pragma unroll
-    for (int s = 0; s < 8; ++s) u[s] = __ldg(src + (size_t)(t + s) * TPR);
+      for (int s = 0; s < 8; ++s) u[s] = __ldg(src + (size_t)(t + s) * TPR);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+      for (int s = 0; s < 8; ++s) {
+        float x[8];
+        unpack8<T>(u[s], x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+      }
+    }
+    for (; t < nt; ++t) {
       float x[8];
-      unpack8<T>(u[s], x);
+      unpack8<T>(__ldg(src + (size_t)t * TPR), x);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
     }
+    float4* dst = reinterpret_cast<float4*>(part + ((size_t)bh * nchunks + chunk) * D + q8 * 8);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
-  for (; t < nt; ++t) {
-    float x[8];
-    unpack8<T>(__ldg(src + (size_t)t * TPR), x);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], x[i]);
+  // the head's last block adds the chunk sums in chunk order
+  __shared__ bool last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&done[bh], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int c = threadIdx.x; c < D; c += 256) {
+    const float* p = part + (size_t)bh * nchunks * D + c;
+    float total = 0.f;
+    for (int ch = 0; ch < nchunks; ++ch) total = __fadd_rn(total, __ldcg(p + (size_t)ch * D));
+    kmean[(size_t)bh * D + c] = __fdiv_rn(total, (float)N);
   }
-  float4* dst = reinterpret_cast<float4*>(part + ((size_t)bh * nchunks + chunk) * D + q8 * 8);
-  dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-}
-
-// K mean, pass 2: chunk sums added in chunk order, then one fp32 division by N.
-// grid (B*H), D threads.
-__global__ void k_mean_finalize(const float* __restrict__ part, int nchunks, int N, int D,
-                                float* __restrict__ kmean) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  const float* p = part + (size_t)bh * nchunks * D + c;
-  float total = 0.f;
-  for (int ch = 0; ch < nchunks; ++ch) total = __fadd_rn(total, p[(size_t)ch * D]);
-  kmean[(size_t)bh * D + c] = __fdiv_rn(total, (float)N);
+  if (threadIdx.x == 0) done[bh] = 0u;
 }
 
 // ---------------------------------------------------------------------------
-// Smoothing + INT4.  grid (NB, B*H, 2): z = 0 quantizes the Q block (after
-// computing its mean), z = 1 the K block (after subtracting kbar).  256 threads.
+// Smoothing + INT4.  grid (NB, B*H, nz): z + zbase = 0 quantizes the Q block
+// (after computing its mean), 1 the K block (after subtracting kbar).  256 threads.
 // FMT: 0 INT4 values as e4m3 codes, 1 INT8 values (the variant), 2 INT4 values
 // packed two per byte (two's-complement nibbles, channel 2c in bits 3:0).
 // Two lanes own one row (16 rows per warp), each half of its channels, so a
@@ -119,14 +128,15 @@ template <typename T, int D, int FMT>
 __global__ void __launch_bounds__(256) k_smooth_quant(
     const T* __restrict__ q, const T* __restrict__ k, int N, long long ldh, int Np, int NB,
     const float* __restrict__ kmean, uint8_t* __restrict__ q_i4, float* __restrict__ q_scale,
-    float* __restrict__ q_mean, uint8_t* __restrict__ k_i4, float* __restrict__ k_scale) {
+    float* __restrict__ q_mean, uint8_t* __restrict__ k_i4, float* __restrict__ k_scale,
+    int zbase) {
   constexpr int RS = 2 * D + 32, HO = D + 16;     // bytes
   constexpr int CPR = D / 8, CPH = CPR / 2;       // 16-byte chunks per row / per half
   constexpr int MH = D / 2 + 4;                   // floats between the two halves of mean
   __shared__ __align__(16) uint8_t tile[128 * RS];
   __shared__ __align__(16) float mean[2 * MH];
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const bool is_q = blockIdx.z == 0;
+  const bool is_q = blockIdx.z + zbase == 0;
   const T* src = is_q ? q : k;
   const int r0 = blk * 128;
   const int nvalid = min(128, N - r0);
@@ -425,29 +435,57 @@ cudaError_t launch_unpack_int4(const uint8_t* packed, uint8_t* codes, size_t byt
 template <typename T, int D>
 cudaError_t launch_qk_corr_t(const QKArgs& a, cudaStream_t st);  // corr.cu
 
+template <typename T, int D, int FMT>
+static void launch_smooth_t(const QKArgs& a, int zbase, int nz, cudaStream_t st) {
+  k_smooth_quant<T, D, FMT><<<dim3(a.NB, a.B * a.H, nz), 256, 0, st>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean,
+      a.q_i4, a.q_scale, a.q_mean, a.k_i4, a.k_scale, zbase);
+}
+
+template <typename T, int D>
+static void launch_smooth(const QKArgs& a, int zbase, int nz, cudaStream_t st) {
+  if (a.qk_bits == 8) launch_smooth_t<T, D, 1>(a, zbase, nz, st);
+  else if (a.packed) launch_smooth_t<T, D, 2>(a, zbase, nz, st);
+  else launch_smooth_t<T, D, 0>(a, zbase, nz, st);
+}
+
+// Two independent chains: K (mean, then smoothing + INT4 of K) and Q
+// (smoothing + INT4 of Q with its block means, then the split of the means
+// and the correction).  With a.side they run concurrently: the Q chain on
+// the library stream, forked from and joined back into `st`.
 template <typename T, int D>
 static cudaError_t launch_qk_t(const QKArgs& a, cudaStream_t st) {
   const int BH = a.B * a.H;
   const int nchunks = a.NB;
   constexpr int WPB = 256 / (D / 8);
-  k_mean_partial<T, D><<<dim3((nchunks + WPB - 1) / WPB, BH), 256, 0, st>>>(
-      static_cast<const T*>(a.k), a.N, a.ldh, nchunks, a.mean_part);
-  k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, nchunks, a.N, D, a.k_mean);
-  if (a.qk_bits == 8)
-    k_smooth_quant<T, D, 1><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
-        a.q_scale, a.q_mean, a.k_i4, a.k_scale);
-  else if (a.packed)
-    k_smooth_quant<T, D, 2><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
-        a.q_scale, a.q_mean, a.k_i4, a.k_scale);
-  else
-    k_smooth_quant<T, D, 0><<<dim3(a.NB, BH, 2), 256, 0, st>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.N, a.ldh, a.Np, a.NB, a.k_mean, a.q_i4,
-        a.q_scale, a.q_mean, a.k_i4, a.k_scale);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaMemsetAsync(a.done, 0, sizeof(unsigned) * BH, st);
   if (e != cudaSuccess) return e;
-  return launch_qk_corr_t<T, D>(a, st);
+  cudaStream_t qs = st;
+  if (a.side) {
+    e = cudaEventRecord(a.fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(a.side, a.fork, 0);
+    if (e != cudaSuccess) return e;
+    qs = a.side;
+  }
+  // K chain
+  k_mean_partial<T, D><<<dim3((nchunks + WPB - 1) / WPB, BH), 256, 0, st>>>(
+      static_cast<const T*>(a.k), a.N, a.ldh, nchunks, a.mean_part, a.done, a.k_mean);
+  if (a.side) {
+    launch_smooth<T, D>(a, 1, 1, st);            // K blocks
+    launch_smooth<T, D>(a, 0, 1, qs);            // Q blocks
+  } else {
+    launch_smooth<T, D>(a, 0, 2, st);            // Q and K blocks in one launch
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // Q chain: the correction needs the block means of Q
+  e = launch_qk_corr_t<T, D>(a, qs);
+  if (e != cudaSuccess) return e;
+  if (a.side && a.join) {                         // (a caller may join later itself)
+    e = cudaEventRecord(a.join, a.side);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, a.join, 0);
+  }
+  return e;
 }
 
 cudaError_t launch_smooth_quant_qk(const QKArgs& a, cudaStream_t st) {
@@ -462,10 +500,11 @@ static cudaError_t launch_v_t(const VArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (a.v_mean) {
     // V smoothing: the per-channel token mean, with the fixed order of the K mean
+    e = cudaMemsetAsync(a.done, 0, sizeof(unsigned) * BH, st);
+    if (e != cudaSuccess) return e;
     constexpr int WPB = 256 / (D / 8);
     k_mean_partial<T, D><<<dim3((a.NB + WPB - 1) / WPB, BH), 256, 0, st>>>(
-        static_cast<const T*>(a.v), a.N, a.ldh, a.NB, a.mean_part);
-    k_mean_finalize<<<BH, D, 0, st>>>(a.mean_part, a.NB, a.N, D, a.v_mean);
+        static_cast<const T*>(a.v), a.N, a.ldh, a.NB, a.mean_part, a.done, a.v_mean);
   }
   k_v_amax<T, D><<<dim3(a.NB, BH), 256, 0, st>>>(static_cast<const T*>(a.v), a.N, a.ldh, a.v_mean,
                                                  a.amax_bits);

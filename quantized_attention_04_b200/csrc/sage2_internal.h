@@ -26,6 +26,11 @@ struct QKArgs {
   int qk_bits;             // 4: INT4 values as e4m3 codes; 8: INT8 values (two's complement)
   int64_t ldh;             // tokens between consecutive heads of q and k (N when contiguous)
   int packed;              // 1 (with qk_bits 4): q_i4/k_i4 hold two INT4 nibbles per byte
+  unsigned* done;          // scratch [B*H]: per-head count of finished K-mean blocks
+  cudaStream_t side;       // non-null: run the Q chain (Q smoothing, q-mean split,
+                           // correction) on this library stream, concurrently with
+                           // the K chain (K mean, K smoothing) on the caller's stream
+  cudaEvent_t fork, join;  // events of that fork / join (with `side`)
 };
 
 struct VArgs {
@@ -38,6 +43,7 @@ struct VArgs {
   float* v_mean;           // nullptr: no V smoothing; else the per-channel token mean [B*H, d]
   float* mean_part;        // scratch [B*H, NB, d] for the V mean (when v_mean is set)
   int64_t ldh;             // tokens between consecutive heads of v (N when contiguous)
+  unsigned* done;          // scratch [B*H] for the V mean (when v_mean is set)
 };
 
 struct AttnArgs {

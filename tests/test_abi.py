@@ -148,7 +148,8 @@ def test_workspace_bytes(L):
         BH = B * H
         parts = [BH * Np * d, BH * Np * d, BH * d * Np, BH * Np * 4, BH * Np * 4,
                  BH * NB * d * 4, BH * d * 4, BH * NB * Np * 4, BH * d * 4, BH * NB * d * 4,
-                 BH * d * 4, 3 * BH * ((NB + 127) // 128) * 128 * d * 2, BH * d * 4]
+                 BH * d * 4, 3 * BH * ((NB + 127) // 128) * 128 * d * 2, BH * d * 4,
+                 2 * BH * 4]
         return sum(up(p) for p in parts)
     for shape in [(1, 2, 256, 64), (2, 8, 2048, 128), (1, 24, 17776, 64), (1, 1, 1, 128)]:
         assert L.sage2_workspace_bytes(*shape) == expect(*shape)
