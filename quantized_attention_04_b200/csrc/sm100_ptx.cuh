@@ -264,25 +264,6 @@ __device__ __forceinline__ void tmem_ld16x256_32(uint32_t taddr, uint32_t (&r)[3
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-// .16x256b.x4: 16 lanes x 32 columns.  Thread t gets, for k = 0..3, the
-// columns 8k + 2(t%4) + {0,1} of lane t/4 (registers 4k, 4k+1) and of lane
-// t/4 + 8 (registers 4k+2, 4k+3) of the 16-lane group at taddr.
-__device__ __forceinline__ void tmem_ld16x256_16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-// .16x256b.x1 store: registers 0, 1 to lane t/4 and 2, 3 to lane t/4 + 8,
-// columns 2(t%4) + {0,1} of the 16-lane group at taddr.
-__device__ __forceinline__ void tmem_st16x256_4(uint32_t taddr, uint32_t r0, uint32_t r1,
-                                                uint32_t r2, uint32_t r3) {
-  asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};"
-               ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2), "r"(r3));
-}
 // .16x256b.x4 store: the mirror of the .16x256b load (registers 4k, 4k+1 to
 // lane t/4, 4k+2, 4k+3 to lane t/4 + 8, columns 8k + 2(t%4) + {0,1}).
 __device__ __forceinline__ void tmem_st16x256_16(uint32_t taddr, const uint32_t (&r)[16]) {
