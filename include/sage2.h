@@ -301,6 +301,26 @@ sage2_status sage2_debug_wait_timeout(sage2_stream_t stream);
  */
 sage2_status sage2_check_device_error(sage2_stream_t stream);
 
+/*
+ * The layout constants of the payloads and of the method as this library
+ * implements them, for callers that produce or consume payloads themselves
+ * (and for tests that check them).  Fills *out; SAGE2_ERR_INVALID_ARG if out
+ * is NULL.  Host only; launches nothing.
+ */
+typedef struct {
+  int version;           /* sage2_version() */
+  int block_rows;        /* query rows per smoothing block and per attention tile (128) */
+  int tile_keys;         /* keys per attention tile: the inner accumulation block (128) */
+  int int4_max;          /* INT4 range [-7, 7] */
+  int int8_max;          /* INT8 variant range [-127, 127] */
+  float p_scale;         /* P~ = e4m3(p_scale * p) */
+  float v_scale_div;     /* v_scale = amax / v_scale_div */
+  int packed_low_first;  /* SAGE2_QK_INT4_PACKED: channel 2c in bits 3:0 of byte c */
+  int key_perm[128];     /* stored k_i4 row n of a 128-row block holds token key_perm[n] */
+  int value_perm[128];   /* v_fp8_t byte p of a 128-token block holds token value_perm[p] */
+} sage2_layout;
+sage2_status sage2_layout_info(sage2_layout* out);
+
 /* Static description of a status code (never NULL). */
 const char* sage2_status_string(sage2_status status);
 

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "sage2_smooth_quant_qk", "sage2_quant_v", "sage2_attn_fwd_quantized", "sage2_attn_fwd",
     "sage2_attn_fwd_noalloc", "sage2_attn_fwd_varlen", "sage2_attn_fwd_host", "sage2_debug_qk_s32", "sage2_workspace_bytes", "sage2_check_device_error",
-    "sage2_status_string", "sage2_version", "attn", "Sage2Error", "lib", "LIB_PATH",
+    "sage2_status_string", "sage2_version", "sage2_layout_info", "attn", "Sage2Error", "lib", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage2.so")
@@ -67,7 +67,14 @@ _SIGS = {
     "sage2_attn_fwd_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sage2_status_string": (ctypes.c_char_p, [_I]),
     "sage2_version": (_I, []),
+    "sage2_layout_info": (_I, [_P]),
 }
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [("version", _I), ("block_rows", _I), ("tile_keys", _I), ("int4_max", _I),
+                ("int8_max", _I), ("p_scale", _F), ("v_scale_div", _F),
+                ("packed_low_first", _I), ("key_perm", _I * 128), ("value_perm", _I * 128)]
 
 
 class Sage2Error(RuntimeError):
@@ -130,6 +137,16 @@ def sage2_status_string(status: int) -> str:
 
 def sage2_version() -> int:
     return int(lib().sage2_version())
+
+
+def sage2_layout_info() -> dict:
+    """The library's layout constants (sage2_layout in include/sage2.h)."""
+    lay = _Layout()
+    _check("sage2_layout_info", lib().sage2_layout_info(ctypes.byref(lay)))
+    d = {name: getattr(lay, name) for name, _ in _Layout._fields_}
+    d["key_perm"] = list(lay.key_perm)
+    d["value_perm"] = list(lay.value_perm)
+    return d
 
 
 def sage2_check_device_error(device=None) -> int:
@@ -271,12 +288,12 @@ attn = sage2_attn_fwd
 def sage2_attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens,
                           causal: bool = False, sm_scale: float | None = None, out_dtype=None,
                           out: torch.Tensor | None = None, qk_bits: int = 4,
-                          smooth_v: bool = False) -> torch.Tensor:
+                          smooth_v: bool = False, packed: bool = False) -> torch.Tensor:
     """Packed variable-length sequences: q, k, v head-major [H, T, d] CUDA
     tensors, cu_seqlens the S+1 token offsets (host ints).  Each sequence is
-    attended within itself; returns o [H, T, d]."""
-    if qk_bits not in _QKF:
-        raise ValueError("qk_bits must be 4 or 8")
+    attended within itself; returns o [H, T, d].  packed stores the INT4
+    payloads two per byte."""
+    fmt = _fmt(qk_bits, packed)
     for t in (q, k, v):
         if t.dim() != 3 or not t.is_cuda or not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous CUDA tensors [H, T, d]")
@@ -291,7 +308,7 @@ def sage2_attn_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_
         out = torch.empty(H, T, d, dtype=out_dtype or q.dtype, device=q.device)
     st = lib().sage2_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), arr, len(cu) - 1, H, T,
                                      d, _DT[q.dtype], _DT[out.dtype], int(bool(causal)),
-                                     float(sm_scale), _QKF[qk_bits], int(bool(smooth_v)),
+                                     float(sm_scale), fmt, int(bool(smooth_v)),
                                      _stream(q))
     _check("sage2_attn_fwd_varlen", st)
     return out
@@ -342,12 +359,11 @@ def sage2_debug_wait_timeout(device=None) -> None:
 
 def sage2_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                         causal: bool = False, sm_scale: float | None = None, qk_bits: int = 4,
-                        smooth_v: bool = False, device=None) -> torch.Tensor:
+                        smooth_v: bool = False, device=None, packed: bool = False) -> torch.Tensor:
     """The forward pass over HOST tensors [B,H,N,d] (pinned for overlap): chunks of
     heads are copied in, run and copied back on library streams joined into the
     current stream of `device`; `out` (host) is complete once that stream is."""
-    if qk_bits not in _QKF:
-        raise ValueError("qk_bits must be 4 or 8")
+    fmt = _fmt(qk_bits, packed)
     for t in (q, k, v, out):
         if t.dim() != 4 or t.is_cuda or not t.is_contiguous():
             raise ValueError("q, k, v, out must be contiguous host tensors [B, H, N, d]")
@@ -363,6 +379,6 @@ def sage2_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: 
     st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     status = lib().sage2_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
                                        _DT[q.dtype], _DT[out.dtype], int(bool(causal)),
-                                       float(sm_scale), _QKF[qk_bits], int(bool(smooth_v)), st)
+                                       float(sm_scale), fmt, int(bool(smooth_v)), st)
     _check("sage2_attn_fwd_host", status)
     return out

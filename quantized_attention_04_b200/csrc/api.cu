@@ -504,4 +504,23 @@ const char* sage2_status_string(sage2_status status) {
 
 int sage2_version(void) { return 100; }
 
+sage2_status sage2_layout_info(sage2_layout* out) {
+  if (!out) return SAGE2_ERR_INVALID_ARG;
+  out->version = sage2_version();
+  out->block_rows = kTile;
+  out->tile_keys = kTile;
+  out->int4_max = 7;
+  out->int8_max = 127;
+  out->p_scale = 448.f;
+  out->v_scale_div = 448.f;
+  out->packed_low_first = 1;
+  for (int j = 0; j < kTile; ++j) {
+    // the quantizer stores token j of a block at row 8*((j/2)%16) + 2*(j/32) + j%2
+    out->key_perm[8 * ((j >> 1) & 15) + 2 * (j >> 5) + (j & 1)] = j;
+    // V^T byte p holds token sigma(p), sigma swapping the 2-bit fields [6:5] and [4:3]
+    out->value_perm[j] = 32 * ((j >> 3) & 3) + 8 * ((j >> 5) & 3) + (j & 7);
+  }
+  return SAGE2_OK;
+}
+
 }  // extern "C"

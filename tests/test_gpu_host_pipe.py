@@ -45,3 +45,20 @@ def test_host_entry_equals_device_entry(qa, cfg, pinned):
                            out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(oh, od.cpu())
+
+
+def test_host_entry_packed_int4_equals_device_entry(qa):
+    """The host-buffer entry with INT4 payloads stored two per byte equals the
+    device entry (INT4 codes) bit for bit."""
+    cfg = CASES[1]
+    q, k, v = make_qkv(cfg)
+    sm = P.default_scale(cfg.d)
+    oh = torch.empty(q.shape, dtype=torch.float32).pin_memory()
+    qa.sage2_attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), oh, causal=cfg.causal,
+                           sm_scale=sm, packed=True)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    od = qa.sage2_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=cfg.causal, sm_scale=sm,
+                           out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, od.cpu())

@@ -70,3 +70,17 @@ def test_varlen_equal_lengths_equal_batched_call(qa):
                             out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(o_var.reshape(H, S, N, d).permute(1, 0, 2, 3), o_b)
+
+
+def test_varlen_packed_int4_equals_int4(qa):
+    """INT4 payloads stored two per byte give the INT4 varlen output bit for bit."""
+    cu = [0, 1, 130, 130, 430, 1458]
+    q, k, v, tdt = packed(cu[-1], 2, 128, "bf16", idx=70)
+    sm = P.default_scale(128)
+    args = (q.cuda(), k.cuda(), v.cuda(), cu)
+    o4 = qa.sage2_attn_fwd_varlen(*args, causal=True, sm_scale=sm, out_dtype=torch.float32)
+    op = qa.sage2_attn_fwd_varlen(*args, causal=True, sm_scale=sm, out_dtype=torch.float32,
+                                  packed=True)
+    torch.cuda.synchronize()
+    assert qa.sage2_check_device_error() == 0
+    assert torch.equal(o4, op)

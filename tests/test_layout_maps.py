@@ -65,3 +65,17 @@ def test_packed_int4_layout_golden():
     bytes (1 | -1 << 4 = 0xF1, 7 | -7 << 4 = 0x97, -8 | 0 = 0x08, 0 | 3 = 0x30)."""
     got = P.pack_int4(np.array([[1, -1, 7, -7, -8, 0, 0, 3]]))
     assert got.tolist() == [[0xF1, 0x97, 0x08, 0x30]]
+
+
+def test_exported_layout_matches_the_documented_orders():
+    """sage2_layout_info() (host only) gives the constants and the two token
+    orders that the GPU payload tests hold the kernels to."""
+    from quantized_attention_04_b200 import build
+    build.build()
+    import quantized_attention_04_b200 as qa
+    lay = qa.sage2_layout_info()
+    assert lay["version"] == qa.sage2_version()
+    assert (lay["block_rows"], lay["tile_keys"], lay["int4_max"], lay["int8_max"]) == (128, 128, 7, 127)
+    assert (lay["p_scale"], lay["v_scale_div"], lay["packed_low_first"]) == (448.0, 448.0, 1)
+    assert lay["key_perm"] == P.key_interleave(128).tolist()
+    assert lay["value_perm"] == P.value_interleave(128).tolist()
