@@ -24,6 +24,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define BM 128
 #define BN 128
@@ -303,7 +306,6 @@ void orc_sage2_head(const float* Q, const float* K, const float* V, int N, int d
 
 int orc_max_threads(void) {
 #ifdef _OPENMP
-  extern int omp_get_max_threads(void);
   return omp_get_max_threads();
 #else
   return 1;
