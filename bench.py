@@ -210,6 +210,8 @@ def oracle_sample(cfg, q, k, v, qk_bits: int = 4):
 
 
 def host_cores() -> int:
+    """Threads the C oracle runs on: OpenMP's default, the host cores this
+    process may use (os.cpu_count() counts every CPU of the machine)."""
     from oracle import c_oracle as corc
     return corc.threads()
 
@@ -236,8 +238,8 @@ def run_reference(args, cfg, world, rank):
         "data": "synthetic (seeded; distributions of the workload)",
         "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
                    "causal": cfg.causal, "input_dtype": cfg.dtype, "sample": desc},
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores,
+                         "host_cpus": os.cpu_count(), "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -368,7 +370,8 @@ def run_sage2(args, cfg, world, rank, local):
             tot_s += dt
             reps += 1
         cpu = {"value": tot_ops / tot_s / 1e12, "unit": "TOPS", "cores": host_cores(),
-               "kind": "oracle", "sample": f"{desc}; {reps} samples", "seconds": tot_s}
+               "host_cpus": os.cpu_count(), "kind": "oracle",
+               "sample": f"{desc}; {reps} samples", "seconds": tot_s}
 
     if rank == 0:
         line = {
