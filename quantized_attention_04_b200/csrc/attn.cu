@@ -45,6 +45,8 @@ namespace sage2 {
 constexpr int kStages = 4;
 constexpr int kSBuf = 3;                         // S tiles in flight in TMEM (P~ of a tile over its S)
 constexpr int kThreads = 512;
+constexpr int kHeadGroup = 8;       // heads whose tiles are interleaved in launch order ...
+constexpr int kGroupMaxTiles = 128; // ... when a head has at most this many query tiles
 constexpr int kSegStride = 36;                   // floats between the 32-key groups in shared memory
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
 constexpr uint32_t kMagicBits = 0x4B400000u;     // 1.5 * 2^23 (INT8 variant, see dequant16)
@@ -224,7 +226,7 @@ __device__ __forceinline__ void store8(void* out, size_t idx, const float (&f)[8
   }
 }
 
-template <int D, int OT, int QB>
+template <int D, int OT, int QB, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
@@ -237,8 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = causal ? (NB - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int bh = blockIdx.y;
+  // Launch order, x fastest.  Plain grid (NB, B*H): one head after another,
+  // its longest query tile (causal) first.  GROUPED grid (G, NB, B*H/G): G
+  // heads round robin, each taking its longest tile first, so that the short
+  // tiles of every head fill the tail of a launch of short heads.
+  const int rank = static_cast<int>(GROUPED ? blockIdx.y : blockIdx.x);
+  const int qt = causal ? (NB - 1 - rank) : rank;
+  const int bh = static_cast<int>(GROUPED ? blockIdx.z * gridDim.x + blockIdx.x : blockIdx.y);
   const int nt = causal ? qt + 1 : NB;           // key tiles this block visits
   const bool tail = (N % 128) != 0;
   volatile int* abort_flag = &sm.abort_flag;
@@ -558,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int OT, int QB>
-static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
+template <int D, int OT, int QB, bool GROUPED>
+static cudaError_t launch_attn_g(const AttnArgs& a, cudaStream_t st, int group) {
   alignas(64) CUtensorMap tq, tk, tv;
   const int BH = a.B * a.H;
   cudaError_t e;
@@ -570,14 +577,27 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
   e = make_tmap_u8_2d(&tv, a.v_fp8_t, static_cast<uint64_t>(BH) * D, a.Np, D, 128);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(AttnSmem<D>) + 1024;
-  e = cudaFuncSetAttribute(k_attn_fwd<D, OT, QB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(k_attn_fwd<D, OT, QB, GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const float L = a.sm_scale * 1.4426950408889634f;
-  k_attn_fwd<D, OT, QB><<<dim3(a.NB, BH), kThreads, smem, st>>>(
+  const dim3 grid = GROUPED ? dim3(group, a.NB, BH / group) : dim3(a.NB, BH);
+  k_attn_fwd<D, OT, QB, GROUPED><<<grid, kThreads, smem, st>>>(
       tq, tk, tv, a.q_scale, a.k_scale, a.qk_corr, a.v_scale, a.v_mean, a.o, a.N, a.ldo, a.Np,
       a.NB, a.causal, L);
   return cudaGetLastError();
+}
+
+// Heads are interleaved (G = the largest divisor of B*H up to kHeadGroup)
+// only when a head has few query tiles, where the tail of the launch is a
+// large share; a long head runs alone, its K and V shared in L2 by every SM.
+template <int D, int OT, int QB>
+static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
+  const int BH = a.B * a.H;
+  int group = kHeadGroup;
+  while (BH % group != 0) --group;
+  if (a.NB <= kGroupMaxTiles && group > 1) return launch_attn_g<D, OT, QB, true>(a, st, group);
+  return launch_attn_g<D, OT, QB, false>(a, st, 1);
 }
 
 template <int QB>

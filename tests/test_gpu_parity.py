@@ -33,6 +33,10 @@ SMALL = [
     small_cfg(1, 64), small_cfg(17, 128, "bf16", True), small_cfg(128, 64, causal=True),
     small_cfg(129, 128), small_cfg(300, 64, "bf16", True), small_cfg(300, 128, causal=True),
     small_cfg(1000, 128, "bf16"), small_cfg(640, 64, causal=False, B=2, H=3),
+    # launch orders: one head after another (B*H = 1, and 11 with no divisor
+    # up to 8) and heads interleaved in groups of 3 (B*H = 9)
+    small_cfg(200, 128, causal=True, H=1), small_cfg(383, 128, "bf16", True, H=11),
+    small_cfg(257, 64, causal=True, B=3, H=3),
 ]
 
 
