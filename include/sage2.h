@@ -229,9 +229,10 @@ sage2_status sage2_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  *                 sequence s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1.
  *   cu_seqlens  : HOST int32 array of S+1 offsets, cu_seqlens[0] = 0,
  *                 non-decreasing, cu_seqlens[S] = T (empty sequences allowed).
- * The sequences run on up to four library-owned streams (longest first, each to
- * the least-loaded one), each with its own workspace for the longest sequence
- * (from the library's pool, as sage2_attn_fwd), forked from and joined back into
+ * The sequences run on four library-owned streams, or up to eight while their
+ * workspaces total at most 4 GiB (longest first, each to the least-loaded one),
+ * each with its own workspace for the longest sequence (from the library's
+ * pool, as sage2_attn_fwd), forked from and joined back into
  * `stream` with events: the call is ordered on `stream` like any other.  Calls
  * on one device are serialised on the host while they enqueue.  Other arguments
  * and statuses as sage2_attn_fwd_ex; a malformed cu_seqlens is

@@ -11,9 +11,10 @@
 // Layout: q, k, v, o are head-major packed, [H, T, d]; sequence s holds tokens
 // cu_seqlens[s] .. cu_seqlens[s+1]-1 of every head.  A sequence is then a
 // [1, H, N_s, d] problem whose heads are T tokens apart, which the kernels
-// take as their head stride.  The sequences are spread over a few library
-// streams (longest first, each to the least-loaded stream), each stream with
-// its own workspace sized for the longest sequence, forked from and joined
+// take as their head stride.  The sequences are spread over 4 library
+// streams, or up to 8 while their workspaces total at most 4 GiB (longest
+// first, each to the least-loaded stream), each stream with its own
+// workspace sized for the longest sequence, forked from and joined
 // back into the caller's stream with events, so that kernels of different
 // sequences fill the GPU together.
 #include <algorithm>
@@ -26,7 +27,9 @@
 
 namespace sage2 {
 
-constexpr int kVarlenStreams = 4;
+constexpr int kVarlenStreams = 8;                        // lanes at most
+constexpr int kVarlenBaseLanes = 4;                      // lanes whatever the workspace size
+constexpr size_t kVarlenLaneBudget = size_t(4) << 30;    // more lanes only within this much workspace
 
 struct VarlenLanes {
   cudaStream_t s[kVarlenStreams] = {};
@@ -101,10 +104,13 @@ extern "C" sage2_status sage2_attn_fwd_varlen(const void* q, const void* k, cons
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return len(a) > len(b); });
   int nlanes = 0;
   for (int s = 0; s < S; ++s) nlanes += len(s) > 0;
-  nlanes = std::min(nlanes, kVarlenStreams);
   if (nlanes == 0) return SAGE2_OK;
-
   const size_t ws_bytes = (layout(gmax, packed_of(qk_format)).total + 255) & ~static_cast<size_t>(255);
+  // short sequences (small workspaces) gain from more lanes; long ones fill
+  // the GPU on their own, and their workspaces are large
+  int cap = kVarlenBaseLanes;
+  while (cap < kVarlenStreams && static_cast<size_t>(cap + 1) * ws_bytes <= kVarlenLaneBudget) ++cap;
+  nlanes = std::min(nlanes, cap);
   uint8_t* ws = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws), ws_bytes * nlanes, pool, st);
   if (e != cudaSuccess) return from_cuda(e);
