@@ -25,6 +25,10 @@ CASES = [
     CONFIGS["C2"],
     Config("host_many_heads", 3, 7, 4000, 64, True, "fp16", q=Dist(1.0), k=Dist(3.0), v=Dist(2.0),
            index=70),
+    # 4 MB heads: 4 heads per 48 MB chunk, so 5 chunks (the last one of 2 heads)
+    # on the 4 library streams, the fifth reusing the first stream's buffers
+    Config("host_chunks", 1, 18, 16384, 128, True, "bf16", q=Dist(1.0), k=Dist(3.0), v=Dist(2.0),
+           index=71),
 ]
 
 
