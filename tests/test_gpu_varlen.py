@@ -84,3 +84,27 @@ def test_varlen_packed_int4_equals_int4(qa):
     torch.cuda.synchronize()
     assert qa.sage2_check_device_error() == 0
     assert torch.equal(o4, op)
+
+
+def test_varlen_many_sequences_equal_per_sequence_calls(qa):
+    """Eleven non-empty sequences of mixed lengths (all eight library streams,
+    some of them twice): each sequence's rows equal the batched call on that
+    sequence alone, bit for bit."""
+    lens = [5, 300, 129, 1, 0, 640, 77, 256, 1000, 33, 512, 128]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    H, d = 2, 64
+    q, k, v, tdt = packed(cu[-1], H, d, "fp16", idx=80)
+    sm = P.default_scale(d)
+    o_var = qa.sage2_attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cu, causal=True, sm_scale=sm,
+                                     out_dtype=torch.float32)
+    for s, n in enumerate(lens):
+        if n == 0:
+            continue
+        sl = lambda t: t[:, cu[s]:cu[s + 1]].unsqueeze(0).contiguous().cuda()
+        o_s = qa.sage2_attn_fwd(sl(q), sl(k), sl(v), causal=True, sm_scale=sm,
+                                out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert torch.equal(o_var[:, cu[s]:cu[s + 1]], o_s[0]), s
+    assert qa.sage2_check_device_error() == 0
