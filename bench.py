@@ -151,25 +151,35 @@ def aggregate(ops_per_rank: float, ms: float, world: int) -> float:
 
 # ---------------------------------------------------------------- recorded DRAM traffic
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "k_attn_fwd_traffic.txt")
-ATTN_SOURCE = os.path.join(ROOT, "quantized_attention_04_b200", "csrc", "attn.cu")
+# every source the attention kernel is compiled from
+ATTN_SOURCES = [os.path.join(ROOT, "quantized_attention_04_b200", "csrc", f)
+                for f in ("attn.cu", "sm100_ptx.cuh", "sage2_internal.h")]
+
+
+def attn_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for path in ATTN_SOURCES:
+        h.update(open(path, "rb").read())
+    return h.hexdigest()
 
 
 def recorded_traffic(workload: str):
     """DRAM bytes (read + write) of one k_attn_fwd launch on `workload`, from
     the ncu record under profiles/, or None when there is none for this
-    workload or the kernel source changed since it was taken (the record
-    carries the SHA-256 of the attention kernel's source)."""
-    import hashlib
+    workload or the kernel's sources changed since it was taken (the record
+    carries the SHA-256 of attn.cu, sm100_ptx.cuh and sage2_internal.h, read
+    in that order)."""
     if not os.path.exists(TRAFFIC_RECORD):
         return None
-    sha = hashlib.sha256(open(ATTN_SOURCE, "rb").read()).hexdigest()
+    sha = attn_sources_sha256()
     rec = {}
     for line in open(TRAFFIC_RECORD):
         line = line.strip()
         if line.startswith("- ") and ":" in line:
             key, val = line[2:].split(":", 1)
             rec[key.strip()] = val.strip().strip("`")
-    if rec.get("workload") != workload or rec.get("attn.cu sha256") != sha:
+    if rec.get("workload") != workload or rec.get("kernel sources sha256") != sha:
         return None
     try:
         return float(rec["dram bytes per launch"])
