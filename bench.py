@@ -56,14 +56,21 @@ def load_peaks():
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms around a
+    timed region (`with ClockSampler(i) as clk: <timed region>`).  Entering
+    waits (at most 5 s) until the sampler has written its first row, so the
+    region cannot end before sampling starts; only rows stamped inside the
+    region are summarised."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    STAMP = "%Y/%m/%d %H:%M:%S.%f"
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -75,27 +82,49 @@ class ClockSampler:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
+        deadline = time.time() + 5.0
+        while self.proc is not None and self.proc.poll() is None and time.time() < deadline:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *exc):
+        self.t1 = time.time()
         if self.proc is not None:
+            time.sleep(0.15)                     # the row that covers the region's end
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
+    @classmethod
+    def parse(cls, lines, t0=None, t1=None):
+        """(sm MHz, max sm MHz, [hw_slowdown, hw_thermal, sw_thermal, sw_power_cap])
+        for each row stamped within [t0, t1 + 0.1 s] (all rows without bounds)."""
+        import datetime
+        rows = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                stamp = datetime.datetime.strptime(parts[0], cls.STAMP).timestamp()
+                row = (float(parts[2]), float(parts[3]), parts[6:10])
+            except ValueError:
+                continue
+            if t0 is not None and not (t0 - 0.1 <= stamp <= t1 + 0.1):
+                continue
+            rows.append(row)
+        return rows
+
     def summary(self):
         rows = []
         if self.path and os.path.exists(self.path):
-            for line in open(self.path):
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-                except ValueError:
-                    continue
+            with open(self.path) as f:
+                rows = self.parse(f, self.t0, self.t1)
             os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
